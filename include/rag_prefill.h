@@ -1,0 +1,210 @@
+/*
+ * rag_prefill.h - C ABI of the precomputed-KV RAG prefill hot path on B200
+ * (sm_100a): paged-pool gather, causal attention of the query block over the
+ * concatenated chunk caches, CacheBlend Impact, and top-k recompute selection.
+ *
+ * Method (cited by page title and section):
+ *   - TurboRAG page, "Technical Details / KV cache precompute": every chunk's
+ *     per-layer K, V are computed once offline (listing `precompute_kv_cache`)
+ *     and reused; at query time K_combined = Concat(K^(1), ..., K^(m), K^(Q))
+ *     and likewise V, in retrieval order, along the sequence axis (listing
+ *     `turborag_inference`).
+ *   - TurboRAG page, "Causal vs non-causal attention":
+ *     Attention(Q, K, V) = softmax(Q K^T / sqrt(d_k) + M_causal) V. Query token
+ *     j of a request sits at position N_doc + j, so every doc key is visible
+ *     to it and the mask is causal only inside the query block.
+ *   - CacheBlend page, "Mathematical formulation": Impact(i) = sum over tokens
+ *     j outside doc(i) of alpha_{j,i}; here j ranges over the query tokens and
+ *     the per-head sums are averaged over the H_q query heads.
+ *   - CacheBlend page, "Recompute ratio trade-off" and the listing
+ *     `select_tokens_for_recompute`: k = max(1, int(N_doc * r)) doc tokens of
+ *     largest Impact.
+ *
+ * Conventions for every entry point:
+ *   - Ownership: the library never allocates or frees device memory. All
+ *     tensors and the workspace belong to the caller; `stream` is a
+ *     cudaStream_t passed as void* (NULL = legacy default stream) and every
+ *     call is asynchronous on it unless stated otherwise.
+ *   - Device pointers must be 16-byte aligned (TMA); strides are implied by
+ *     the shapes (dense, row-major, innermost dimension last).
+ *   - Argument, shape and dtype errors are reported synchronously by the
+ *     return value and nothing is launched. Problems the device finds (a page
+ *     id outside the pool, a chunk whose page count is not ceil(len / 16), a
+ *     pipeline wait that gave up) are recorded in the workspace error word,
+ *     never trapped, and reported by rag_last_device_error.
+ *   - Indices of doc tokens are logical positions within their request,
+ *     0 .. N_doc,b - 1, in concatenation order.
+ */
+#ifndef RAG_PREFILL_H_
+#define RAG_PREFILL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define RAG_API __attribute__((visibility("default")))
+#else
+#define RAG_API
+#endif
+
+#define RAG_ABI_VERSION 1
+#define RAG_PAGE_SIZE 16
+
+typedef enum {
+  RAG_OK = 0,
+  RAG_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad scalar            */
+  RAG_ERR_SHAPE = 2,       /* inconsistent sizes                              */
+  RAG_ERR_PAGE_OOB = 3,    /* device: a page id outside [0, num_pages)        */
+  RAG_ERR_UNSUPPORTED = 4, /* valid request this build does not implement      */
+  RAG_ERR_CUDA = 5,        /* a CUDA runtime call failed                      */
+  RAG_ERR_TIMEOUT = 6,     /* device: a pipeline wait gave up                 */
+  RAG_ERR_WORKSPACE = 7,   /* workspace missing or smaller than required      */
+  RAG_ERR_GEOMETRY = 8     /* device: chunk pages do not match its length     */
+} rag_status;
+
+typedef enum { RAG_BF16 = 0, RAG_F32 = 1 } rag_dtype;
+
+/* The paged pool of precomputed chunk caches (caller-owned device memory).
+ * k, v: [num_layers][num_pages][num_kv_heads][16][head_dim] of `dtype`.
+ * Page p of layer l, kv head g holds 16 consecutive tokens of one chunk.
+ * Supported: RAG_BF16 with head_dim 128 (tensor-core path), RAG_F32 with
+ * head_dim 64 or 128 (CUDA-core path). */
+typedef struct {
+  void* k;
+  void* v;
+  int32_t num_layers;
+  int32_t num_pages;
+  int32_t num_kv_heads;
+  int32_t page_size; /* must be RAG_PAGE_SIZE */
+  int32_t head_dim;
+  int32_t dtype;     /* rag_dtype */
+} rag_kv_pool;
+
+/* One batch of B requests. The int32 arrays are DEVICE pointers; the scalars
+ * are host-side totals and maxima used to size launches and the workspace.
+ * Request b retrieved the chunk-list entries [req_chunk_off[b],
+ * req_chunk_off[b+1]) in retrieval order; an entry may repeat a chunk.
+ *   req_chunk_off  [B+1]  prefix over requests of chunk-list entries
+ *   chunk_doc_off  [C+1]  prefix over the chunk list of chunk lengths (tokens)
+ *   chunk_page_off [C+1]  prefix over the chunk list of page counts; entry c
+ *                         must have ceil(len_c / 16) pages
+ *   page_ids       [P]    physical page of each referenced page, in order
+ *   q_off          [B+1]  prefix over requests of query tokens
+ * Request b's doc tokens are chunk_doc_off[req_chunk_off[b]] ..
+ * chunk_doc_off[req_chunk_off[b+1]] - 1; its query tokens are q_off[b] ..
+ * q_off[b+1] - 1. */
+typedef struct {
+  int32_t num_requests;  /* B, 0 .. 4096 */
+  int32_t num_chunks;    /* C */
+  int32_t num_page_refs; /* P */
+  int32_t total_q;       /* q_off[B] */
+  int32_t total_doc;     /* chunk_doc_off[C] */
+  int32_t max_q;         /* max_b query tokens */
+  int32_t max_doc;       /* max_b doc tokens */
+  int32_t max_pages;     /* max_b pages referenced by one request */
+  const int32_t* req_chunk_off;
+  const int32_t* chunk_doc_off;
+  const int32_t* chunk_page_off;
+  const int32_t* page_ids;
+  const int32_t* q_off;
+} rag_batch;
+
+/* ABI version of the loaded library (RAG_ABI_VERSION). */
+RAG_API int32_t rag_abi_version(void);
+
+/* Static text for a rag_status value. */
+RAG_API const char* rag_status_string(int32_t status);
+
+/* Number of SMs of the current device (launch sizing). */
+RAG_API int32_t rag_num_sms(void);
+
+/* Pool write (TurboRAG page, "Technical Details / KV cache precompute"; the
+ * listing `precompute_kv_cache`): store one chunk's dense K, V
+ * [n_tokens][num_kv_heads][head_dim] (pool dtype, device) into the pages
+ * page_ids[0 .. n_pages-1] (device int32) of `layer`. Token t goes to page
+ * page_ids[t / 16], slot t % 16; the slots of the last page beyond n_tokens
+ * are zeroed. n_pages must equal ceil(n_tokens / 16). A page id outside the
+ * pool is skipped and sets RAG_ERR_PAGE_OOB's bit in *device_err (optional
+ * device int32, may be NULL). */
+RAG_API rag_status rag_kv_pool_write(const rag_kv_pool* pool, int32_t layer, const int32_t* page_ids, int32_t n_pages,
+                             int32_t n_tokens, const void* k, const void* v, int32_t* device_err, void* stream);
+
+/* Bytes of workspace rag_fused_prefill_attn needs for this pool, batch and
+ * head count (0 on invalid arguments). The workspace holds the device error
+ * word, per-row softmax statistics and split-KV partials; it must be zeroed
+ * once before first use (rag_workspace_init) and may be reused across calls
+ * on one stream. */
+RAG_API size_t rag_workspace_size(const rag_kv_pool* pool, const rag_batch* batch, int32_t num_q_heads);
+
+/* Clear the workspace's error word (async on `stream`). */
+RAG_API rag_status rag_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Fused prefill of one layer for the whole batch:
+ *   gather [K_1; ...; K_m; K_q] through the page table (TurboRAG page,
+ *   Concat equation), then for every query head h (KV head h / G) and query
+ *   token j of request b:  O[j,h] = sum_i softmax_i(scale * Q[j,h] . K_i) V_i
+ *   over keys i <= N_doc,b + j (TurboRAG page, causal attention equation).
+ * q      [total_q][num_q_heads][head_dim]   pool dtype, device
+ * kq, vq [total_q][num_kv_heads][head_dim]  the query block's own K, V
+ * sm_scale <= 0 selects 1 / sqrt(head_dim).
+ * o      [total_q][num_q_heads][head_dim]   output, pool dtype
+ * row_lse optional [total_q][num_q_heads] fp32: log sum_i exp(scale Q.K_i)
+ * impact  optional [total_doc + total_q] fp32 output. When given, the call
+ *   also computes CacheBlend's Impact (CacheBlend page, "Mathematical
+ *   formulation"): for request b the segment at offset
+ *   chunk_doc_off[req_chunk_off[b]] + q_off[b] holds, for each of its
+ *   N_doc,b + q_b key positions i, (1/H_q) sum_h sum_j alpha^h_{j,i}; the doc
+ *   part comes first. The impacts of a request's segment add up to q_b.
+ *   Pass it on the layer whose attention selects tokens (the last layer).
+ * workspace: device, >= rag_workspace_size() bytes, 256-byte aligned. */
+RAG_API rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch, const void* q,
+                                  int32_t num_q_heads, const void* kq, const void* vq, float sm_scale, void* o,
+                                  float* row_lse, float* impact, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* Recompute count for a request with n_doc doc tokens (CacheBlend page,
+ * "Recompute ratio trade-off" and listing): max(1, int(n_doc * r)) with the
+ * product in double precision, and 0 when n_doc is 0. Host function. */
+RAG_API int32_t rag_recompute_count(int32_t n_doc, double r);
+
+/* Top-k recompute selection for every request (CacheBlend listing
+ * `select_tokens_for_recompute`, torch.topk over the doc slice):
+ * impact   as written by rag_fused_prefill_attn (device fp32)
+ * r        recompute ratio, 0 < r < 1
+ * k_cap    row length of the outputs, >= rag_recompute_count(max_doc, r),
+ *          <= 8192
+ * topk_idx [B][k_cap] int32 device output: the k_b doc positions of largest
+ *          impact ordered by (impact descending, position ascending); the
+ *          rest of the row is -1
+ * topk_val optional [B][k_cap] fp32: their impacts (0 past k_b)
+ * k_out    optional [B] int32: k_b */
+RAG_API rag_status rag_impact_topk(const float* impact, const rag_batch* batch, double r, int32_t k_cap,
+                           int32_t* topk_idx, float* topk_val, int32_t* k_out, void* stream);
+
+/* Synchronise `stream`, read and clear the workspace error word. Returns
+ * RAG_OK when the device reported nothing, else the most severe of
+ * RAG_ERR_TIMEOUT, RAG_ERR_PAGE_OOB, RAG_ERR_GEOMETRY; *bits (optional)
+ * receives the raw bits (1 page, 2 geometry, 4 timeout). */
+RAG_API rag_status rag_last_device_error(void* workspace, int32_t* bits, void* stream);
+
+/* Kernel launches this library has made in this process (all entry points). */
+RAG_API int64_t rag_launch_count(void);
+
+/* Per-kernel timing: when enabled, every launch is bracketed by CUDA events
+ * on its stream. rag_profile_collect synchronises, writes the summed device
+ * milliseconds and launch counts per kernel kind (0 pool write, 1 attention,
+ * 2 split combine, 3 impact, 4 top-k, 5 fp32 attention, 6 fp32 impact) into
+ * the first n_kinds entries of ms and launches (either may be NULL), and
+ * resets the record. */
+RAG_API void rag_profile_enable(int32_t on);
+RAG_API rag_status rag_profile_collect(double* ms, int64_t* launches, int32_t n_kinds);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RAG_PREFILL_H_ */

@@ -1,0 +1,595 @@
+// Attention pass of the fused prefill: the query block of each request
+// attends over [K_1; ...; K_m; K_q] gathered from the paged pool
+// (TurboRAG page, "Technical Details": Concat of the per-chunk caches and the
+// query's own K/V; causal attention softmax(QK^T/sqrt(d_k) + M_causal) V).
+//
+// One persistent CTA per SM walks work items (request, kv head, 128-row tile,
+// split of the key tiles). Rows pack the G query heads of one KV head with
+// the query tokens (row = token * G + head-in-group), so GQA groups share
+// every K/V tile in the MMA M dimension. Per 128-key tile:
+//   K producer warp : page table -> 8 TMA page boxes (or one box of K_q)
+//   V producer warp : the same for V
+//   MMA warp        : S = Q K^T (tcgen05, smem x smem -> TMEM), then
+//                     O += P V (tcgen05, P from TMEM x V from smem)
+//   4 softmax warps : thread = row = TMEM lane; mask, online max/sum in the
+//                     log2 domain, P (bf16) back to TMEM, lazy O rescale
+// S and P are double-buffered in TMEM so QK^T of tile t+1 overlaps the
+// softmax of tile t. Every wait is bounded; a timeout raises a device error.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "params.cuh"
+
+namespace rag {
+
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kDescSlots = 4;
+constexpr int kTileBytes = kBN * kHeadDim * 2;   // one K or V tile, bf16
+constexpr int kHalfBytes = kTileBytes / 2;       // 64 columns of d
+constexpr int kQBytes = kBM * kHeadDim * 2;
+constexpr int kFwdThreads = 224;                 // 4 softmax + K + V + MMA warps
+constexpr float kRescaleThreshold = 8.0f;        // log2 units: rescale O when the max grows by > 2^8
+
+// TMEM columns
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+
+struct TileDesc {
+  int32_t kind;       // 0: doc tile from the pool, 1: query-key tile
+  int32_t kbase;      // query tile: index of its first query key
+  uint8_t nvalid[kPagesPerTile];
+};
+
+
+struct FwdCtrl {
+  uint64_t q_full, q_empty;
+  uint64_t kfull[kKStages], kempty[kKStages];
+  uint64_t vfull[kVStages], vempty[kVStages];
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t o_free, teardown;
+  uint64_t desc_full[kDescSlots], desc_empty[kDescSlots];
+  TileDesc desc[kDescSlots];
+  uint32_t tmem_base;
+  int32_t abort;
+  int32_t total_items;
+};
+
+constexpr size_t kFwdSmemData = kQBytes + size_t(kKStages + kVStages) * kTileBytes;
+
+__host__ size_t fwd_smem_bytes(int num_requests) {
+  return 1024 + kFwdSmemData + sizeof(FwdCtrl) + sizeof(int32_t) * (num_requests + 1) + 64;
+}
+
+struct FwdItem {
+  int b, g, rt, split;
+  int t_begin, t_end;   // tiles of the unit handled by this item
+  int n_doc_tiles;
+  ReqInfo req;
+};
+
+__device__ __forceinline__ FwdItem decode_fwd_item(const FwdParams& p, const int32_t* prefix, int w) {
+  const int B = p.batch.num_requests;
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {  // last b with prefix[b] <= w
+    int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= w) lo = mid; else hi = mid - 1;
+  }
+  FwdItem it;
+  it.b = lo;
+  it.req = load_req(p.batch, lo);
+  const FwdShape sh = fwd_shape(p.batch, it.req, p.group, p.tiles_per_split);
+  int local = w - prefix[lo];
+  it.rt = local % sh.n_rt;
+  local /= sh.n_rt;
+  it.split = local % sh.n_split;
+  it.g = local / sh.n_split;
+  it.n_doc_tiles = doc_tiles(it.req);
+  const int last_tok = min(it.req.n_q, (it.rt + 1) * kBM / p.group) - 1;
+  const int n_tiles = it.n_doc_tiles + query_tiles_upto(last_tok);
+  it.t_begin = min(it.split * p.tiles_per_split, n_tiles);
+  it.t_end = min(it.t_begin + p.tiles_per_split, n_tiles);
+  return it;
+}
+
+__device__ __forceinline__ void raise_abort(FwdCtrl* c, int32_t* err) {
+  if (!c->abort) {
+    atomicOr(err, kDevErrTimeout);
+    c->abort = 1;
+  }
+}
+
+// Wait bounded by time only (teardown after an abort).
+__device__ __forceinline__ void wait_quiet(uint64_t* bar, uint32_t parity) {
+  int zero = 0;
+  mbar_wait(bar, parity, &zero);
+}
+
+// K-major, 128B-swizzled tile of 128 rows x 128 bf16 stored as two 64-column
+// halves of 16 KB; k-step kk covers columns [16 kk, 16 kk + 16).
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk) {
+  return sdesc_sw128(base + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
+}
+// V tile [128 keys][128 d] as the B operand with N = d contiguous (MN-major):
+// k-step kk covers keys [16 kk, 16 kk + 16); the two 64-wide d halves are
+// 16 KB apart (leading byte offset), 8-key groups 1 KB apart (stride).
+__device__ __forceinline__ uint64_t v_desc(uint32_t base, int kk) {
+  return sdesc_sw128(base + kk * 16 * 128, kHalfBytes, 1024);
+}
+
+__global__ void __launch_bounds__(kFwdThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kq,
+                const __grid_constant__ CUtensorMap tm_vq, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + kQBytes;
+  uint8_t* sV = sK + kKStages * kTileBytes;
+  FwdCtrl* ctl = reinterpret_cast<FwdCtrl*>(sV + kVStages * kTileBytes);
+  int32_t* prefix = reinterpret_cast<int32_t*>(ctl + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int B = p.batch.num_requests;
+  const int G = p.group;
+
+  // zero the impact accumulator for the impact pass that follows
+  if (p.impact_zero) {
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + tid; i < p.impact_len;
+         i += int64_t(gridDim.x) * blockDim.x)
+      p.impact_zero[i] = 0.f;
+  }
+
+  if (tid == 0) {
+    mbar_init(&ctl->q_full, 1);
+    mbar_init(&ctl->q_empty, 1);
+    for (int s = 0; s < kKStages; ++s) { mbar_init(&ctl->kfull[s], 1); mbar_init(&ctl->kempty[s], 1); }
+    for (int s = 0; s < kVStages; ++s) { mbar_init(&ctl->vfull[s], 1); mbar_init(&ctl->vempty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ctl->s_full[s], 1);
+      mbar_init(&ctl->p_full[s], 128);
+      mbar_init(&ctl->pv_done[s], 1);
+    }
+    mbar_init(&ctl->o_free, 128);
+    mbar_init(&ctl->teardown, 1);
+    for (int s = 0; s < kDescSlots; ++s) { mbar_init(&ctl->desc_full[s], 1); mbar_init(&ctl->desc_empty[s], 4); }
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 6) {
+    tmem_alloc(&ctl->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_kq);
+  }
+  if (warp == 5 && lane == 0) { tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_vq); }
+
+  // per-request item counts -> exclusive prefix (warp 0), total in ctl
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < B; base += 32) {
+      const int b = base + lane;
+      int cnt = 0;
+      if (b < B) {
+        const ReqInfo r = load_req(p.batch, b);
+        if (!req_ok(p.batch, r) && blockIdx.x == 0) atomicOr(p.err, kDevErrGeometry);
+        const FwdShape sh = fwd_shape(p.batch, r, G, p.tiles_per_split);
+        cnt = p.num_kv_heads * sh.n_split * sh.n_rt;
+      }
+      int incl = cnt;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (b < B) prefix[b] = carry + incl - cnt;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      // more work than the workspace was sized for: descriptors disagree with
+      // the host totals; report and do nothing
+      if (carry > p.max_items) {
+        if (blockIdx.x == 0) atomicOr(p.err, kDevErrGeometry);
+        carry = 0;
+        for (int b = 0; b < B; ++b) prefix[b] = 0;
+      }
+      prefix[B] = carry;
+      ctl->total_items = carry;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (blockIdx.x == 0 && p.item_prefix) {
+    for (int b = tid; b <= B; b += blockDim.x) p.item_prefix[b] = prefix[b];
+  }
+
+  const int total_items = ctl->total_items;
+  const uint32_t tmem = ctl->tmem_base;
+  volatile int* abort_flag = &ctl->abort;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ softmax
+    const int r = tid;
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    uint32_t t_glob = 0;
+    int bad = 0;
+    for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
+      const FwdItem it = decode_fwd_item(p, prefix, w);
+      const int n = it.t_end - it.t_begin;
+      const int pr = it.rt * kBM + r;
+      const int tok = pr / G;
+      const int head = it.g * G + (pr % G);
+      const bool row_valid = tok < it.req.n_q;
+      float m_ref = -INFINITY, l_sum = 0.f;
+      for (int i = 0; i < n; ++i) {
+        const uint32_t t = t_glob + i;
+        const uint32_t buf = t & 1;
+        const uint32_t slot = t % kDescSlots;
+        if (!mbar_wait(&ctl->desc_full[slot], (t / kDescSlots) & 1, abort_flag)) { bad = 1; break; }
+        const TileDesc td = ctl->desc[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->desc_empty[slot]);
+        if (!mbar_wait(&ctl->s_full[buf], (t >> 1) & 1, abort_flag)) { bad = 1; break; }
+        tc_fence_after();
+        float x[kBN];
+        {
+          uint32_t u[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            tmem_ld32(tmem + lane_off + (buf ? kColS1 : kColS0) + 32 * c, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[32 * c + j] = __uint_as_float(u[j]);
+          }
+        }
+        // mask and move to the log2 domain
+        float mx = -INFINITY;
+        if (td.kind == 0) {
+          uint32_t nv_lo = *reinterpret_cast<const uint32_t*>(&td.nvalid[0]);
+          uint32_t nv_hi = *reinterpret_cast<const uint32_t*>(&td.nvalid[4]);
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) {
+            const int pg = c >> 4;
+            const uint32_t nv = ((pg < 4 ? nv_lo >> (8 * pg) : nv_hi >> (8 * (pg - 4))) & 0xffu);
+            const float v = (uint32_t(c & 15) < nv) ? x[c] * p.scale_log2 : -INFINITY;
+            x[c] = v;
+            mx = fmaxf(mx, v);
+          }
+        } else {
+          const int lim = tok - td.kbase;   // keys c <= lim are visible
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) {
+            const float v = (c <= lim) ? x[c] * p.scale_log2 : -INFINITY;
+            x[c] = v;
+            mx = fmaxf(mx, v);
+          }
+        }
+        float alpha = 1.f;
+        bool need = false;
+        if (i == 0) {
+          m_ref = mx;
+        } else if (mx > m_ref + kRescaleThreshold) {
+          alpha = ex2(m_ref - mx);
+          need = true;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          // O must hold PV of the previous tile before it is rescaled
+          const uint32_t tp = t - 1;
+          if (!mbar_wait(&ctl->pv_done[tp & 1], (tp >> 1) & 1, abort_flag)) { bad = 1; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t u[32];
+            tmem_ld32(tmem + lane_off + kColO + 32 * c, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * alpha);
+            tmem_st32(tmem + lane_off + kColO + 32 * c, u);
+          }
+          tmem_wait_st();
+          if (need) { l_sum *= alpha; m_ref = mx; }
+        }
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        // P buffer `buf` was last read by PV of tile t - 2
+        if (t >= 2) {
+          const uint32_t tq = t - 2;
+          if (!mbar_wait(&ctl->pv_done[buf], (tq >> 1) & 1, abort_flag)) { bad = 1; break; }
+        }
+        float ls = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float a = ex2(x[64 * h + 2 * j] - m_use);
+            const float b2 = ex2(x[64 * h + 2 * j + 1] - m_use);
+            ls += a + b2;
+            pk[j] = pack_bf16x2(a, b2);
+          }
+          tmem_st32(tmem + lane_off + (buf ? kColP1 : kColP0) + 32 * h, pk);
+        }
+        l_sum += ls;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&ctl->p_full[buf]);
+      }
+      if (bad) break;
+      t_glob += n;
+
+      // ---- epilogue: O of this item
+      float o[kHeadDim];
+      if (n > 0) {
+        const uint32_t tl = t_glob - 1;
+        if (!mbar_wait(&ctl->pv_done[tl & 1], (tl >> 1) & 1, abort_flag)) { bad = 1; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_off + kColO + 32 * c, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[32 * c + j] = __uint_as_float(u[j]);
+        }
+        tc_fence_before();
+        mbar_arrive(&ctl->o_free);
+      } else {
+#pragma unroll
+        for (int j = 0; j < kHeadDim; ++j) o[j] = 0.f;
+      }
+      if (p.direct) {
+        if (row_valid) {
+          const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+          const int64_t row = int64_t(it.req.q0 + tok) * p.num_q_heads + head;
+          uint4* dst = reinterpret_cast<uint4*>(p.o + row * kHeadDim);
+#pragma unroll
+          for (int c = 0; c < kHeadDim / 8; ++c) {
+            uint4 v;
+            v.x = pack_bf16x2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
+            v.y = pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
+            v.z = pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
+            v.w = pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
+            dst[c] = v;
+          }
+          const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+          p.row_m2[row] = m_use;
+          p.row_il[row] = l_sum > 0.f ? 1.f / (l_sum * float(p.num_q_heads)) : 0.f;
+          if (p.row_lse) p.row_lse[row] = (m_use + __log2f(l_sum)) * 0.69314718055994531f;
+        }
+      } else {
+        float4* dst = reinterpret_cast<float4*>(p.part + (size_t(w) * kBM + r) * kPartStride);
+#pragma unroll
+        for (int c = 0; c < kHeadDim / 4; ++c) dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        dst[kHeadDim / 4] = make_float4(m_ref, l_sum, 0.f, 0.f);
+      }
+    }
+    if (bad) raise_abort(ctl, p.err);
+  } else if (warp == 4 || warp == 5) {
+    // ------------------------------------------------------------ producers
+    const bool is_k = (warp == 4);
+    const CUtensorMap* tm_pool = is_k ? &tm_k : &tm_v;
+    const CUtensorMap* tm_qkv = is_k ? &tm_kq : &tm_vq;
+    uint8_t* sbase = is_k ? sK : sV;
+    const int nstages = is_k ? kKStages : kVStages;
+    uint64_t* full = is_k ? ctl->kfull : ctl->vfull;
+    uint64_t* empty = is_k ? ctl->kempty : ctl->vempty;
+    uint32_t t_glob = 0, q_iter = 0;
+    int bad = 0;
+    for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
+      const FwdItem it = decode_fwd_item(p, prefix, w);
+      const int n = it.t_end - it.t_begin;
+      if (n == 0) continue;
+      if (is_k) {
+        if (q_iter > 0 && !mbar_wait(&ctl->q_empty, (q_iter - 1) & 1, abort_flag)) { bad = 1; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&ctl->q_full, kQBytes);
+          const int tok0 = it.req.q0 + it.rt * (kBM / G);
+          tma_load_3d(sQ, &tm_q, &ctl->q_full, 0, it.g * G, tok0);
+          tma_load_3d(sQ + kHalfBytes, &tm_q, &ctl->q_full, 64, it.g * G, tok0);
+        }
+        ++q_iter;
+      }
+      for (int i = 0; i < n; ++i) {
+        const uint32_t t = t_glob + i;
+        const int tile = it.t_begin + i;
+        const bool doc = tile < it.n_doc_tiles;
+        PageRef pg;
+        pg.page = -1; pg.nvalid = 0; pg.lstart = 0;
+        if (doc && lane < kPagesPerTile)
+          pg = page_ref(p.batch, it.req, tile * kPagesPerTile + lane, p.num_pages, is_k ? p.err : nullptr);
+        if (is_k) {
+          const uint32_t slot = t % kDescSlots;
+          if (t >= kDescSlots && !mbar_wait(&ctl->desc_empty[slot], ((t / kDescSlots) - 1) & 1, abort_flag)) {
+            bad = 1;
+            break;
+          }
+          TileDesc* d = &ctl->desc[slot];
+          if (doc) {
+            if (lane < kPagesPerTile) d->nvalid[lane] = uint8_t(pg.nvalid);
+            if (lane == 0) { d->kind = 0; d->kbase = 0; }
+          } else if (lane == 0) {
+            d->kind = 1;
+            d->kbase = (tile - it.n_doc_tiles) * kBN;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->desc_full[slot]);
+        }
+        const int s = t % nstages;
+        if (t >= uint32_t(nstages) && !mbar_wait(&empty[s], ((t / nstages) - 1) & 1, abort_flag)) {
+          bad = 1;
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], kTileBytes);
+        __syncwarp();
+        uint8_t* dst = sbase + s * kTileBytes;
+        if (doc) {
+          if (lane < kPagesPerTile) {
+            const int row = pg.page >= 0
+                                ? ((p.layer * p.num_pages + pg.page) * p.num_kv_heads + it.g) * kPage
+                                : -kPage;   // fully out of range: the box is zero-filled
+            tma_load_2d(dst + lane * kPage * 128, tm_pool, &full[s], 0, row);
+            tma_load_2d(dst + kHalfBytes + lane * kPage * 128, tm_pool, &full[s], 64, row);
+          }
+        } else if (lane == 0) {
+          const int kq0 = it.req.q0 + (tile - it.n_doc_tiles) * kBN;
+          tma_load_3d(dst, tm_qkv, &full[s], 0, it.g, kq0);
+          tma_load_3d(dst + kHalfBytes, tm_qkv, &full[s], 64, it.g, kq0);
+        }
+      }
+      t_glob += n;
+    }
+    if (bad) {
+      raise_abort(ctl, p.err);
+    }
+    // let every copy this warp issued land before the CTA exits
+    if (lane == 0) {
+      const uint32_t issued = t_glob;
+      const uint32_t first = issued > uint32_t(nstages) ? issued - nstages : 0;
+      if (ctl->abort)
+        for (uint32_t t = first; t < issued; ++t) wait_quiet(&full[t % nstages], (t / nstages) & 1);
+      if (is_k && ctl->abort && q_iter > 0) wait_quiet(&ctl->q_full, (q_iter - 1) & 1);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0);
+      const uint32_t idesc_pv = idesc_bf16_f32(kBM, kHeadDim, 1);
+      const uint32_t q_base = smem_u32(sQ);
+      uint32_t t_glob = 0, q_iter = 0, o_uses = 0;
+      int bad = 0;
+      for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
+        const FwdItem it = decode_fwd_item(p, prefix, w);
+        const int n = it.t_end - it.t_begin;
+        if (n == 0) continue;
+        if (!mbar_wait(&ctl->q_full, q_iter & 1, abort_flag)) { bad = 1; break; }
+        tc_fence_after();
+        for (int i = 0; i <= n && !bad; ++i) {
+          if (i < n) {
+            const uint32_t t = t_glob + i;
+            const int s = t % kKStages;
+            if (!mbar_wait(&ctl->kfull[s], (t / kKStages) & 1, abort_flag)) { bad = 1; break; }
+            tc_fence_after();
+            const uint32_t k_base = smem_u32(sK + s * kTileBytes);
+            const uint32_t d_s = tmem + ((t & 1) ? kColS1 : kColS0);
+#pragma unroll
+            for (int kk = 0; kk < kHeadDim / 16; ++kk)
+              mma_ss(d_s, kmajor_desc(q_base, kk), kmajor_desc(k_base, kk), idesc_qk, kk > 0);
+            tc_commit(&ctl->s_full[t & 1]);
+            tc_commit(&ctl->kempty[s]);
+          }
+          if (i >= 1) {
+            const uint32_t tp = t_glob + i - 1;
+            const int sv = tp % kVStages;
+            if (i == 1) {
+              if (o_uses > 0 && !mbar_wait(&ctl->o_free, (o_uses - 1) & 1, abort_flag)) { bad = 1; break; }
+              ++o_uses;
+            }
+            if (!mbar_wait(&ctl->p_full[tp & 1], (tp >> 1) & 1, abort_flag)) { bad = 1; break; }
+            if (!mbar_wait(&ctl->vfull[sv], (tp / kVStages) & 1, abort_flag)) { bad = 1; break; }
+            tc_fence_after();
+            const uint32_t v_base = smem_u32(sV + sv * kTileBytes);
+            const uint32_t a_p = tmem + ((tp & 1) ? kColP1 : kColP0);
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk)
+              mma_ts(tmem + kColO, a_p + kk * 8, v_desc(v_base, kk), idesc_pv, (i > 1) || (kk > 0));
+            tc_commit(&ctl->pv_done[tp & 1]);
+            tc_commit(&ctl->vempty[sv]);
+          }
+        }
+        if (bad) break;
+        tc_commit(&ctl->q_empty);
+        t_glob += n;
+        ++q_iter;
+      }
+      if (bad) raise_abort(ctl, p.err);
+      // every MMA issued so far completes before TMEM is released
+      tc_commit(&ctl->teardown);
+      wait_quiet(&ctl->teardown, 0);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 6) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- combine
+
+
+// Merge the split partials (O, m, l) of one (request, kv head, row tile):
+// m = max_s m_s, l = sum_s l_s 2^(m_s - m), O = sum_s O_s 2^(m_s - m) / l.
+// grid: x = kv head * max row tiles + row tile, y = request; 8 warps, warp per row.
+__global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p, int max_rt) {
+  const int b = blockIdx.y;
+  const int g = blockIdx.x / max_rt;
+  const int rt = blockIdx.x % max_rt;
+  const ReqInfo req = load_req(p.batch, b);
+  const FwdShape sh = fwd_shape(p.batch, req, p.group, p.tiles_per_split);
+  if (rt >= sh.n_rt || g >= p.num_kv_heads) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.group;
+  const int base = p.item_prefix[b];
+  for (int r = warp; r < kBM; r += 8) {
+    const int pr = rt * kBM + r;
+    const int tok = pr / G;
+    if (tok >= req.n_q) break;
+    const int head = g * G + pr % G;
+    float m = -INFINITY;
+    for (int s = 0; s < sh.n_split; ++s) {
+      const size_t slot = size_t(base) + (size_t(g) * sh.n_split + s) * sh.n_rt + rt;
+      if (slot >= size_t(p.max_items) || size_t(base) >= size_t(p.item_prefix[p.batch.num_requests])) return;
+      m = fmaxf(m, p.part[(slot * kBM + r) * kPartStride + kHeadDim]);
+    }
+    const float m_use = (m == -INFINITY) ? 0.f : m;
+    float l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < sh.n_split; ++s) {
+      const size_t slot = size_t(base) + (size_t(g) * sh.n_split + s) * sh.n_rt + rt;
+      const float* pr_row = p.part + (slot * kBM + r) * kPartStride;
+      const float ms = pr_row[kHeadDim];
+      const float ls = pr_row[kHeadDim + 1];
+      const float wgt = (ms == -INFINITY) ? 0.f : ex2(ms - m_use);
+      l += ls * wgt;
+      const float4 v = reinterpret_cast<const float4*>(pr_row)[lane];
+      acc.x += v.x * wgt; acc.y += v.y * wgt; acc.z += v.z * wgt; acc.w += v.w * wgt;
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const int64_t row = int64_t(req.q0 + tok) * p.num_q_heads + head;
+    uint2 out;
+    out.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    out.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(p.o + row * kHeadDim)[lane] = out;
+    if (lane == 0) {
+      p.row_m2[row] = m_use;
+      p.row_il[row] = l > 0.f ? 1.f / (l * float(p.num_q_heads)) : 0.f;
+      if (p.row_lse) p.row_lse[row] = (m_use + __log2f(l)) * 0.69314718055994531f;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- launchers
+
+cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tkq, const CUtensorMap& tvq, const FwdParams& p, int grid,
+                            cudaStream_t stream) {
+  const size_t smem = fwd_smem_bytes(p.batch.num_requests);
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  attn_fwd_kernel<<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, tkq, tvq, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_combine(const CombineParams& p, int max_rt, int num_requests, cudaStream_t stream) {
+  dim3 grid(p.num_kv_heads * max_rt, num_requests);
+  attn_combine_kernel<<<grid, 256, 0, stream>>>(p, max_rt);
+  return cudaGetLastError();
+}
+
+}  // namespace rag

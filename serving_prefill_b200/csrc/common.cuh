@@ -1,0 +1,171 @@
+// Shared device-side definitions: batch geometry, work decomposition and the
+// workspace layout used by the attention, combine, impact and top-k kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace rag {
+
+constexpr int kPage = 16;             // tokens per pool page
+constexpr int kHeadDim = 128;         // head_dim of the tensor-core path
+constexpr int kBM = 128;              // attention rows (query token x head-in-group) per tile
+constexpr int kBN = 128;              // keys per tile
+constexpr int kPagesPerTile = kBN / kPage;
+constexpr int kImpactRows = 256;      // rows per impact-pass block (MMA N)
+constexpr int kMaxRequests = 4096;
+constexpr int kPartStride = 132;      // floats per partial row: O[128], m, l, pad
+
+// device error word bits (rag_last_device_error reports them)
+enum : int32_t {
+  kDevErrPage = 1,       // a page id outside [0, num_pages)
+  kDevErrGeometry = 2,   // a chunk whose page count is not ceil(len / 16)
+  kDevErrTimeout = 4,    // a pipeline wait gave up
+};
+
+struct BatchDev {
+  const int32_t* req_chunk_off;    // [B+1]
+  const int32_t* chunk_doc_off;    // [C+1]
+  const int32_t* chunk_page_off;   // [C+1]
+  const int32_t* page_ids;         // [num_page_refs]
+  const int32_t* q_off;            // [B+1]
+  int32_t num_requests;
+  // host-side totals and maxima; a request that breaks them is skipped and
+  // reported (kDevErrGeometry) so that no kernel reads or writes out of range
+  int32_t num_chunks, num_page_refs, total_q, total_doc, max_q, max_pages, max_doc;
+};
+
+struct ReqInfo {
+  int32_t c0, c1;       // chunk-list entries of the request
+  int32_t doc0, n_doc;  // first doc token (over the batch) and doc tokens
+  int32_t p0, n_pages;  // first page reference and pages
+  int32_t q0, n_q;      // first query token and query tokens
+};
+
+__device__ __forceinline__ ReqInfo load_req(const BatchDev& B, int b) {
+  ReqInfo r;
+  r.c0 = __ldg(B.req_chunk_off + b);
+  r.c1 = __ldg(B.req_chunk_off + b + 1);
+  r.doc0 = __ldg(B.chunk_doc_off + r.c0);
+  r.n_doc = __ldg(B.chunk_doc_off + r.c1) - r.doc0;
+  r.p0 = __ldg(B.chunk_page_off + r.c0);
+  r.n_pages = __ldg(B.chunk_page_off + r.c1) - r.p0;
+  r.q0 = __ldg(B.q_off + b);
+  r.n_q = __ldg(B.q_off + b + 1) - r.q0;
+  return r;
+}
+
+// A request whose descriptor entries stay inside the host-declared sizes.
+__device__ __forceinline__ bool req_ok(const BatchDev& B, const ReqInfo& r) {
+  return r.c0 >= 0 && r.c0 <= r.c1 && r.c1 <= B.num_chunks && r.p0 >= 0 && r.n_pages >= 0 &&
+         r.p0 + r.n_pages <= B.num_page_refs && r.n_pages <= B.max_pages && r.q0 >= 0 && r.n_q >= 0 &&
+         r.q0 + r.n_q <= B.total_q && r.n_q <= B.max_q && r.doc0 >= 0 && r.n_doc >= 0 &&
+         r.doc0 + r.n_doc <= B.total_doc && r.n_doc <= B.max_doc && r.n_doc <= r.n_pages * kPage;
+}
+
+__host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Tiles of one request: ceil(pages / 8) doc tiles in page-list order, then
+// the query block's keys in tiles of 128.
+__device__ __forceinline__ int doc_tiles(const ReqInfo& r) { return ceil_div(r.n_pages, kPagesPerTile); }
+
+// Attention work units: (request, kv head, 128-row tile, split of the key tiles).
+struct FwdShape {
+  int n_rt, n_split;
+};
+__device__ __forceinline__ FwdShape fwd_shape(const BatchDev& B, const ReqInfo& r, int G, int tiles_per_split) {
+  FwdShape s;
+  if (r.n_q <= 0 || !req_ok(B, r)) { s.n_rt = 0; s.n_split = 0; return s; }
+  s.n_rt = ceil_div(r.n_q * G, kBM);
+  s.n_split = ceil_div(doc_tiles(r) + ceil_div(r.n_q, kBN), tiles_per_split);
+  return s;
+}
+
+// Query-key tiles that a block of rows ending at token `last_tok` can see.
+__device__ __forceinline__ int query_tiles_upto(int last_tok) { return last_tok / kBN + 1; }
+
+// Impact work units: (request, kv head, 256-row block, split of key tiles).
+__device__ __forceinline__ FwdShape impact_shape(const BatchDev& B, const ReqInfo& r, int G,
+                                                int tiles_per_split) {
+  FwdShape s;
+  if (r.n_q <= 0 || !req_ok(B, r)) { s.n_rt = 0; s.n_split = 0; return s; }
+  s.n_rt = ceil_div(r.n_q * G, kImpactRows);
+  s.n_split = ceil_div(doc_tiles(r) + ceil_div(r.n_q, kBN), tiles_per_split);
+  return s;
+}
+
+// Locate the chunk of global page reference `gref` inside chunk-list range
+// [c0, c1): the last c with chunk_page_off[c] <= gref.
+__device__ __forceinline__ int chunk_of_page(const BatchDev& B, int c0, int c1, int gref) {
+  int lo = c0, hi = c1 - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(B.chunk_page_off + mid) <= gref) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// One page of a doc tile: where it lives and which of its slots are real.
+struct PageRef {
+  int32_t page;     // physical page, or -1 when absent/invalid
+  int32_t nvalid;   // valid slots (0..16)
+  int32_t lstart;   // logical doc position of slot 0 within the request
+};
+
+__device__ __forceinline__ PageRef page_ref(const BatchDev& B, const ReqInfo& r, int ref, int num_pages,
+                                            int32_t* err) {
+  PageRef p;
+  p.page = -1; p.nvalid = 0; p.lstart = 0;
+  if (ref >= r.n_pages) return p;
+  const int gref = r.p0 + ref;
+  const int c = chunk_of_page(B, r.c0, r.c1, gref);
+  const int cp0 = __ldg(B.chunk_page_off + c), cp1 = __ldg(B.chunk_page_off + c + 1);
+  const int k = gref - cp0;
+  const int cstart = __ldg(B.chunk_doc_off + c);
+  const int len = __ldg(B.chunk_doc_off + c + 1) - cstart;
+  if (k < 0 || gref >= cp1 || len < 0 || cstart < r.doc0 || cstart + len > r.doc0 + r.n_doc) {
+    if (err) atomicOr(err, kDevErrGeometry);
+    return p;
+  }
+  int nv = len - k * kPage;
+  if (nv <= 0 || (gref == cp1 - 1 && nv > kPage)) {
+    if (err) atomicOr(err, kDevErrGeometry);
+  }
+  nv = nv < 0 ? 0 : (nv > kPage ? kPage : nv);
+  const int page = __ldg(B.page_ids + gref);
+  if (page < 0 || page >= num_pages) {
+    if (err) atomicOr(err, kDevErrPage);
+    return p;
+  }
+  p.page = page;
+  p.nvalid = nv;
+  p.lstart = cstart - r.doc0 + k * kPage;
+  return p;
+}
+
+// Workspace layout (bytes, each region 256-aligned):
+//   [0, 256)                   error word and flags
+//   item prefix                (kMaxRequests + 1) int32
+//   row_m2                     total_q * H_q fp32   (reference max, log2 units)
+//   row_il                     total_q * H_q fp32   (1 / (l * H_q))
+//   partials                   items * 128 * kPartStride fp32
+struct WsLayout {
+  size_t off_prefix, off_m2, off_il, off_part, total;
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+__host__ __device__ inline WsLayout ws_layout(int64_t total_q, int num_q_heads, int64_t max_items) {
+  WsLayout w;
+  size_t at = 256;
+  w.off_prefix = at; at = align256(at + sizeof(int32_t) * (kMaxRequests + 1));
+  w.off_m2 = at; at = align256(at + sizeof(float) * size_t(total_q) * num_q_heads);
+  w.off_il = at; at = align256(at + sizeof(float) * size_t(total_q) * num_q_heads);
+  w.off_part = at; at = align256(at + sizeof(float) * size_t(max_items) * kBM * kPartStride);
+  w.total = at;
+  return w;
+}
+
+}  // namespace rag

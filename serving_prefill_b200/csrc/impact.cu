@@ -1,0 +1,367 @@
+// Impact pass (CacheBlend page, "Mathematical formulation": Impact(i) is the
+// sum of the normalised attention weights alpha_{j,i} that tokens outside
+// doc(i) give to token i; the `select_tokens_for_recompute` listing sums the
+// query rows of the softmax over each column).
+//
+// alpha_{j,i} = exp(s_{j,i} - m_j) / l_j needs each row's final max and sum,
+// which the attention pass leaves in (row_m2, row_il). This pass recomputes
+// the scores in transposed form, S^T = K Q^T, so that a TMEM lane is a key:
+// each thread sums its key's weights over up to 256 query rows with no
+// cross-thread reduction, then adds the total into impact[] with one atomic.
+//
+//   producer warp : Q rows of the block (TMA, once per item) and K tiles
+//                   gathered through the page table (TMA page boxes)
+//   MMA warp      : S^T (128 keys x N rows) = K (smem) x Q^T (smem) -> TMEM
+//   4 epilogue warps: exp2 / scale / accumulate per key, atomicAdd
+// Impact is averaged over the H_q query heads (1/H_q is folded into row_il),
+// so the impacts of all N_doc + q columns of a request add up to q.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "params.cuh"
+
+namespace rag {
+
+constexpr int kIKStages = 4;
+constexpr int kIDescSlots = 6;
+constexpr int kITileBytes = kBN * kHeadDim * 2;     // K tile
+constexpr int kIHalf = kITileBytes / 2;
+constexpr int kIQHalf = kImpactRows * 128;          // 256 rows x 64 d (bf16) per d-half
+constexpr int kIQBytes = 2 * kIQHalf;
+constexpr int kImpThreads = 192;
+
+struct ImpDesc {
+  int32_t kind;      // 0 doc tile, 1 query-key tile
+  int32_t kbase;
+  uint8_t nvalid[kPagesPerTile];
+  int32_t lstart[kPagesPerTile];
+};
+
+
+struct ImpCtrl {
+  uint64_t q_full, q_empty;
+  uint64_t kfull[kIKStages], kempty[kIKStages];
+  uint64_t s_full[2], s_free[2];
+  uint64_t teardown;
+  uint64_t desc_full[kIDescSlots], desc_empty[kIDescSlots];
+  ImpDesc desc[kIDescSlots];
+  float2 mi[kImpactRows];
+  uint32_t tmem_base;
+  int32_t abort;
+  int32_t total_items;
+};
+
+__host__ size_t impact_smem_bytes(int num_requests) {
+  return 1024 + kIQBytes + size_t(kIKStages) * kITileBytes + sizeof(ImpCtrl) +
+         sizeof(int32_t) * (num_requests + 1) + 64;
+}
+
+struct ImpItem {
+  int b, g, rb, split, t_begin, t_end, n_doc_tiles, nrows, N;
+  ReqInfo req;
+};
+
+__device__ __forceinline__ ImpItem decode_imp_item(const ImpactParams& p, const int32_t* prefix, int w) {
+  const int B = p.batch.num_requests;
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= w) lo = mid; else hi = mid - 1;
+  }
+  ImpItem it;
+  it.b = lo;
+  it.req = load_req(p.batch, lo);
+  const FwdShape sh = impact_shape(p.batch, it.req, p.group, p.tiles_per_split);
+  int local = w - prefix[lo];
+  it.rb = local % sh.n_rt;
+  local /= sh.n_rt;
+  it.split = local % sh.n_split;
+  it.g = local / sh.n_split;
+  it.n_doc_tiles = doc_tiles(it.req);
+  const int G = p.group;
+  const int last_tok = min(it.req.n_q, (it.rb + 1) * kImpactRows / G) - 1;
+  const int n_tiles = it.n_doc_tiles + query_tiles_upto(last_tok);
+  it.t_begin = min(it.split * p.tiles_per_split, n_tiles);
+  it.t_end = min(it.t_begin + p.tiles_per_split, n_tiles);
+  it.nrows = min(kImpactRows, it.req.n_q * G - it.rb * kImpactRows);
+  it.N = (it.nrows + 31) & ~31;
+  return it;
+}
+
+__device__ __forceinline__ uint64_t imp_kdesc(uint32_t base, int kk) {
+  return sdesc_sw128(base + (kk >> 2) * kIHalf + (kk & 3) * 32, 16, 1024);
+}
+__device__ __forceinline__ uint64_t imp_qdesc(uint32_t base, int kk) {
+  return sdesc_sw128(base + (kk >> 2) * kIQHalf + (kk & 3) * 32, 16, 1024);
+}
+
+__device__ __forceinline__ void imp_abort(ImpCtrl* c, int32_t* err) {
+  if (!c->abort) {
+    atomicOr(err, kDevErrTimeout);
+    c->abort = 1;
+  }
+}
+
+__global__ void __launch_bounds__(kImpThreads, 1)
+impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_kq, const ImpactParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + kIQBytes;
+  ImpCtrl* ctl = reinterpret_cast<ImpCtrl*>(sK + kIKStages * kITileBytes);
+  int32_t* prefix = reinterpret_cast<int32_t*>(ctl + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int B = p.batch.num_requests;
+  const int G = p.group;
+
+  if (tid == 0) {
+    mbar_init(&ctl->q_full, 1);
+    mbar_init(&ctl->q_empty, 1);
+    for (int s = 0; s < kIKStages; ++s) { mbar_init(&ctl->kfull[s], 1); mbar_init(&ctl->kempty[s], 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&ctl->s_full[s], 1); mbar_init(&ctl->s_free[s], 128); }
+    mbar_init(&ctl->teardown, 1);
+    for (int s = 0; s < kIDescSlots; ++s) { mbar_init(&ctl->desc_full[s], 1); mbar_init(&ctl->desc_empty[s], 4); }
+    ctl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&ctl->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) { tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_kq); }
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < B; base += 32) {
+      const int b = base + lane;
+      int cnt = 0;
+      if (b < B) {
+        const ReqInfo r = load_req(p.batch, b);
+        if (!req_ok(p.batch, r) && blockIdx.x == 0) atomicOr(p.err, kDevErrGeometry);
+        const FwdShape sh = impact_shape(p.batch, r, G, p.tiles_per_split);
+        cnt = p.num_kv_heads * sh.n_split * sh.n_rt;
+      }
+      int incl = cnt;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (b < B) prefix[b] = carry + incl - cnt;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) { prefix[B] = carry; ctl->total_items = carry; }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const int total_items = ctl->total_items;
+  const uint32_t tmem = ctl->tmem_base;
+  volatile int* abort_flag = &ctl->abort;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ epilogue: thread = key
+    const int k = tid;
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    uint32_t t_glob = 0;
+    int bad = 0;
+    for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
+      const ImpItem it = decode_imp_item(p, prefix, w);
+      const int n = it.t_end - it.t_begin;
+      if (n == 0) continue;
+      named_bar_sync(1, 128);
+      for (int r = tid; r < kImpactRows; r += 128) {
+        float2 v = make_float2(INFINITY, 0.f);
+        if (r < it.nrows) {
+          const int pr = it.rb * kImpactRows + r;
+          const int64_t row = int64_t(it.req.q0 + pr / G) * p.num_q_heads + it.g * G + pr % G;
+          v = make_float2(p.row_m2[row], p.row_il[row]);
+        }
+        ctl->mi[r] = v;
+      }
+      named_bar_sync(1, 128);
+      float* seg = p.impact + (it.req.doc0 + it.req.q0);
+      for (int i = 0; i < n; ++i) {
+        const uint32_t t = t_glob + i;
+        const uint32_t buf = t & 1;
+        const uint32_t slot = t % kIDescSlots;
+        if (!mbar_wait(&ctl->desc_full[slot], (t / kIDescSlots) & 1, abort_flag)) { bad = 1; break; }
+        const ImpDesc* d = &ctl->desc[slot];
+        const int kind = d->kind;
+        bool valid;
+        int lpos, rlim = 0;
+        if (kind == 0) {
+          const int pg = k >> 4, sl = k & 15;
+          valid = sl < int(d->nvalid[pg]);
+          lpos = d->lstart[pg] + sl;
+        } else {
+          const int kq = d->kbase + k;
+          valid = kq < it.req.n_q;
+          lpos = it.req.n_doc + kq;
+          rlim = kq * G - it.rb * kImpactRows;   // rows r >= rlim see this key
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->desc_empty[slot]);
+        if (!mbar_wait(&ctl->s_full[buf], (t >> 1) & 1, abort_flag)) { bad = 1; break; }
+        tc_fence_after();
+        float acc = 0.f;
+        const uint32_t col = tmem + lane_off + (buf ? 256u : 0u);
+        for (int c = 0; c < it.N; c += 32) {
+          uint32_t u[32];
+          tmem_ld32(col + c, u);
+          tmem_wait_ld();
+          if (kind == 0) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float2 mi = ctl->mi[c + j];
+              acc += ex2(__uint_as_float(u[j]) * p.scale_log2 - mi.x) * mi.y;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float2 mi = ctl->mi[c + j];
+              const float pv = ex2(__uint_as_float(u[j]) * p.scale_log2 - mi.x) * mi.y;
+              acc += (c + j >= rlim) ? pv : 0.f;
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&ctl->s_free[buf]);
+        if (valid) atomicAdd(seg + lpos, acc);
+      }
+      t_glob += n;
+    }
+    if (bad) imp_abort(ctl, p.err);
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    uint32_t t_glob = 0, q_iter = 0;
+    int bad = 0;
+    for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
+      const ImpItem it = decode_imp_item(p, prefix, w);
+      const int n = it.t_end - it.t_begin;
+      if (n == 0) continue;
+      if (q_iter > 0 && !mbar_wait(&ctl->q_empty, (q_iter - 1) & 1, abort_flag)) { bad = 1; break; }
+      if (lane == 0) {
+        const int nbox = (it.N + kBM - 1) / kBM;
+        mbar_arrive_expect_tx(&ctl->q_full, nbox * 2 * (kBM * 128));
+        for (int bi = 0; bi < nbox; ++bi) {
+          const int tok0 = it.req.q0 + (it.rb * kImpactRows + bi * kBM) / G;
+          tma_load_3d(sQ + bi * (kBM * 128), &tm_q, &ctl->q_full, 0, it.g * G, tok0);
+          tma_load_3d(sQ + kIQHalf + bi * (kBM * 128), &tm_q, &ctl->q_full, 64, it.g * G, tok0);
+        }
+      }
+      ++q_iter;
+      for (int i = 0; i < n; ++i) {
+        const uint32_t t = t_glob + i;
+        const int tile = it.t_begin + i;
+        const bool doc = tile < it.n_doc_tiles;
+        PageRef pg;
+        pg.page = -1; pg.nvalid = 0; pg.lstart = 0;
+        if (doc && lane < kPagesPerTile)
+          pg = page_ref(p.batch, it.req, tile * kPagesPerTile + lane, p.num_pages, p.err);
+        const uint32_t slot = t % kIDescSlots;
+        if (t >= kIDescSlots && !mbar_wait(&ctl->desc_empty[slot], ((t / kIDescSlots) - 1) & 1, abort_flag)) {
+          bad = 1;
+          break;
+        }
+        ImpDesc* d = &ctl->desc[slot];
+        if (doc) {
+          if (lane < kPagesPerTile) { d->nvalid[lane] = uint8_t(pg.nvalid); d->lstart[lane] = pg.lstart; }
+          if (lane == 0) { d->kind = 0; d->kbase = 0; }
+        } else if (lane == 0) {
+          d->kind = 1;
+          d->kbase = (tile - it.n_doc_tiles) * kBN;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->desc_full[slot]);
+        const int s = t % kIKStages;
+        if (t >= uint32_t(kIKStages) && !mbar_wait(&ctl->kempty[s], ((t / kIKStages) - 1) & 1, abort_flag)) {
+          bad = 1;
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(&ctl->kfull[s], kITileBytes);
+        __syncwarp();
+        uint8_t* dst = sK + s * kITileBytes;
+        if (doc) {
+          if (lane < kPagesPerTile) {
+            const int row = pg.page >= 0 ? ((p.layer * p.num_pages + pg.page) * p.num_kv_heads + it.g) * kPage
+                                         : -kPage;
+            tma_load_2d(dst + lane * kPage * 128, &tm_k, &ctl->kfull[s], 0, row);
+            tma_load_2d(dst + kIHalf + lane * kPage * 128, &tm_k, &ctl->kfull[s], 64, row);
+          }
+        } else if (lane == 0) {
+          const int kq0 = it.req.q0 + (tile - it.n_doc_tiles) * kBN;
+          tma_load_3d(dst, &tm_kq, &ctl->kfull[s], 0, it.g, kq0);
+          tma_load_3d(dst + kIHalf, &tm_kq, &ctl->kfull[s], 64, it.g, kq0);
+        }
+      }
+      t_glob += n;
+    }
+    if (bad) imp_abort(ctl, p.err);
+    if (lane == 0 && ctl->abort) {
+      int zero = 0;
+      const uint32_t first = t_glob > uint32_t(kIKStages) ? t_glob - kIKStages : 0;
+      for (uint32_t t = first; t < t_glob; ++t) mbar_wait(&ctl->kfull[t % kIKStages], (t / kIKStages) & 1, &zero);
+      if (q_iter > 0) mbar_wait(&ctl->q_full, (q_iter - 1) & 1, &zero);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t q_base = smem_u32(sQ);
+      uint32_t t_glob = 0, q_iter = 0;
+      int bad = 0;
+      for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
+        const ImpItem it = decode_imp_item(p, prefix, w);
+        const int n = it.t_end - it.t_begin;
+        if (n == 0) continue;
+        const uint32_t idesc = idesc_bf16_f32(kBN, it.N, 0);
+        if (!mbar_wait(&ctl->q_full, q_iter & 1, abort_flag)) { bad = 1; break; }
+        tc_fence_after();
+        for (int i = 0; i < n; ++i) {
+          const uint32_t t = t_glob + i;
+          const int s = t % kIKStages;
+          if (!mbar_wait(&ctl->kfull[s], (t / kIKStages) & 1, abort_flag)) { bad = 1; break; }
+          if (t >= 2 && !mbar_wait(&ctl->s_free[t & 1], ((t - 2) >> 1) & 1, abort_flag)) { bad = 1; break; }
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(sK + s * kITileBytes);
+          const uint32_t d_s = tmem + ((t & 1) ? 256u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kHeadDim / 16; ++kk)
+            mma_ss(d_s, imp_kdesc(k_base, kk), imp_qdesc(q_base, kk), idesc, kk > 0);
+          tc_commit(&ctl->s_full[t & 1]);
+          tc_commit(&ctl->kempty[s]);
+        }
+        if (bad) break;
+        tc_commit(&ctl->q_empty);
+        t_glob += n;
+        ++q_iter;
+      }
+      if (bad) imp_abort(ctl, p.err);
+      tc_commit(&ctl->teardown);
+      int zero = 0;
+      mbar_wait(&ctl->teardown, 0, &zero);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_impact(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tkq,
+                          const ImpactParams& p, int grid, cudaStream_t stream) {
+  const size_t smem = impact_smem_bytes(p.batch.num_requests);
+  cudaError_t e = cudaFuncSetAttribute(impact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  impact_kernel<<<grid, kImpThreads, smem, stream>>>(tq, tk, tkq, p);
+  return cudaGetLastError();
+}
+
+}  // namespace rag

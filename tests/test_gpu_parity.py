@@ -1,0 +1,147 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Sizes span several 128-key tiles, several 128-row tiles, ragged chunk tails,
+several requests, GQA groups of 1 to 8, split and unsplit key ranges, and the
+edge cases of the method (one query token, one-token chunks, a request with
+no query tokens, repeated chunks). The full-size workloads run in the launch
+configuration the benchmark times.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.prefill as orc
+from workloads import get_workload, make_layout, scaled
+
+from gpu_support import DeviceCase, assert_impact_close, check_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def small_cases():
+    l2 = get_workload("llama2_7b_l1")
+    l3 = get_workload("llama3_8b_l32")
+    b16 = get_workload("batched16")
+    l70 = get_workload("long70b")
+    return {
+        "tiny": get_workload("tiny"),
+        "tiny_f32_gqa": scaled(get_workload("tiny"), num_q_heads=8, num_kv_heads=2, head_dim=128,
+                               chunk_lens=(33, 1, 16, 70), q_len=13),
+        "mha_ragged": scaled(l2, num_q_heads=4, num_kv_heads=4, chunk_lens=(200, 77, 300), q_len=40),
+        "gqa4_rows3": scaled(l3, num_layers=2, num_q_heads=16, num_kv_heads=4,
+                             chunk_lens=(333, 129, 500, 17), q_len=70),
+        "pooled": scaled(b16, num_q_heads=8, num_kv_heads=2, n_requests=5, n_pool_chunks=12,
+                         chunk_len_range=(1, 400), chunks_per_req=(1, 4), q_range=(1, 90)),
+        "g8_long_rows": scaled(l70, num_q_heads=16, num_kv_heads=2, chunk_lens=(700,) * 6, q_len=150),
+        "one_query_token": scaled(l2, num_q_heads=8, num_kv_heads=8, chunk_lens=(1, 15, 16, 17, 129), q_len=1),
+        "query_longer_than_tile": scaled(l3, num_layers=1, num_q_heads=4, num_kv_heads=2, chunk_lens=(60,),
+                                         q_len=300),
+    }
+
+
+CASES = small_cases()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_parity_small(name):
+    w = CASES[name]
+    layers = list(range(w.num_layers))
+    case = DeviceCase(w, layers=layers)
+    for layer in layers:
+        check_layer(case, layer, with_impact=(layer == w.impact_layer_index))
+
+
+@pytest.mark.parametrize("name", ["tiny", "pooled", "gqa4_rows3"])
+def test_pool_write_bit_exact(name):
+    w = CASES[name]
+    case = DeviceCase(w, layers=[0])
+    ref = orc.run_workload_layer(case.lay, case.inputs[0], want_impact=False, keep_pool=True)
+    view = torch.int16 if w.dtype == "bf16" else torch.int32
+    bits = np.uint16 if w.dtype == "bf16" else np.uint32
+    gk = case.pool.k[0].contiguous().view(view).cpu().numpy().view(bits)
+    gv = case.pool.v[0].contiguous().view(view).cpu().numpy().view(bits)
+    assert np.array_equal(gk, ref.pool_k[0]) and np.array_equal(gv, ref.pool_v[0])
+    assert int(case.err.item()) == 0
+
+
+def test_physical_page_permutation_is_bit_identical():
+    w = CASES["pooled"]
+    lay = make_layout(w)
+    a = DeviceCase(w, lay=lay, layers=[0]).run_layer(0, True)
+    b = DeviceCase(w, lay=lay.with_page_permutation(seed=11), layers=[0]).run_layer(0, True)
+    assert np.array_equal(a["o"], b["o"])
+    assert np.array_equal(a["lse"], b["lse"])
+    assert np.array_equal(a["topk_idx"], b["topk_idx"])
+    np.testing.assert_allclose(a["impact"], b["impact"], rtol=1e-6)
+
+
+def test_chunk_order_permutes_impact():
+    w = CASES["mha_ragged"]
+    lay = make_layout(w)
+    order = [2, 0, 1]
+    lay2 = lay.with_chunk_order([order])
+    a = DeviceCase(w, lay=lay, layers=[0]).run_layer(0, True)
+    b = DeviceCase(w, lay=lay2, layers=[0]).run_layer(0, True)
+    np.testing.assert_allclose(a["o"], b["o"], atol=2e-2, rtol=2e-2)
+    starts1 = np.cumsum([0] + [lay.chunk_len[c] for c in lay.req_chunks[0]])
+    starts2 = np.cumsum([0] + [lay2.chunk_len[c] for c in lay2.req_chunks[0]])
+    for pos2, c in enumerate(lay2.req_chunks[0]):
+        pos1 = lay.req_chunks[0].index(c)
+        n = lay.chunk_len[c]
+        assert_impact_close(b["impact"][starts2[pos2]:starts2[pos2] + n], a["impact"][starts1[pos1]:starts1[pos1] + n])
+
+
+def test_request_without_query_tokens():
+    w = scaled(get_workload("batched16"), num_q_heads=8, num_kv_heads=2, n_requests=3, n_pool_chunks=5,
+               chunk_len_range=(20, 200), chunks_per_req=(1, 3), q_range=(1, 40))
+    lay = make_layout(w)
+    lay.q_lens[1] = 0
+    from workloads.rag import _flatten
+    _flatten(lay)
+    case = DeviceCase(w, lay=lay, layers=[0])
+    out, ref = check_layer(case, 0, with_impact=True)
+    n0 = lay.doc_lens[0] + lay.q_lens[0]
+    assert np.all(out["impact"][n0:n0 + lay.doc_lens[1]] == 0)
+
+
+def test_impact_total_is_query_length():
+    w = CASES["pooled"]
+    case = DeviceCase(w, layers=[0])
+    out = case.run_layer(0, True)
+    at = 0
+    for b in range(case.lay.num_requests):
+        n = case.lay.doc_lens[b] + case.lay.q_lens[b]
+        np.testing.assert_allclose(out["impact"][at:at + n].sum(), case.lay.q_lens[b], rtol=1e-4)
+        at += n
+
+
+def test_run_twice_is_deterministic_for_o():
+    w = CASES["g8_long_rows"]
+    case = DeviceCase(w, layers=[0])
+    a = case.run_layer(0, False)
+    b = case.run_layer(0, False)
+    assert np.array_equal(a["o"], b["o"]) and np.array_equal(a["lse"], b["lse"])
+
+
+# ------------------------------------------------------------------ full size
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["tiny", "llama2_7b_l1", "batched16", "long70b"])
+def test_parity_full_size(name):
+    w = get_workload(name)
+    case = DeviceCase(w, layers=[w.impact_layer_index])
+    check_layer(case, w.impact_layer_index, with_impact=True)
+
+
+@pytest.mark.slow
+def test_parity_full_size_32_layers():
+    """All 32 layers run as the benchmark runs them; layers 0 and 31 (impact) are checked."""
+    w = get_workload("llama3_8b_l32")
+    case = DeviceCase(w)
+    for layer in range(w.num_layers):
+        q, kq, vq = case.dev_inputs[layer]
+        case.engine.attend(layer, q, kq, vq, with_impact=False)
+    torch.cuda.synchronize()
+    check_layer(case, 0, with_impact=False)
+    check_layer(case, w.num_layers - 1, with_impact=True)
