@@ -1,0 +1,511 @@
+"""Benchmark of the fused precomputed-KV RAG prefill step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl mine|reference]
+
+A step is one pass of the whole hot path over one batch: the fused attention
+of every layer of the workload (paged gather + causal attention), Impact on
+the selecting layer, and the top-k recompute selection. The metric is doc-KV
+tokens per second (the doc tokens whose cached K/V the step consumes), over
+all GPUs. Inputs are seeded synthetic tensors shaped like the pages'
+workloads (see workloads/rag.py); the precomputed pool is resident in HBM.
+
+L2 policy: the timed steps rotate over enough independent copies of the
+inputs (pool, Q, K_q, V_q, workspace) that each step's working set has left
+the 126 MB L2 before it is touched again. Each copy's step is captured once
+in a CUDA graph and replayed.
+
+One JSON line is printed by rank 0. With --impl reference the same metric is
+measured for the fp64 CPU oracle on the host cores (a bounded sample per step).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import get_workload, make_layer_inputs, make_layout  # noqa: E402
+
+DEFAULT_CONFIG = "llama2_7b_l1"
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "doc-KV tokens/s through fused attn+impact+top-k; % of roofline at 1 B200"
+
+
+# ----------------------------------------------------------------------------- arithmetic of the roofline
+
+def step_work(w, lay):
+    """Algorithmic FLOPs and bytes of one step (method's own work, once)."""
+    d, hq, hk, eb = w.head_dim, w.num_q_heads, w.num_kv_heads, w.elem_bytes
+    pairs = sum(q * n + q * (q + 1) // 2 for q, n in zip(lay.q_lens, lay.doc_lens))
+    attn_flops = 4 * d * hq * pairs                           # QK^T and PV per visible pair
+    impact_flops = 2 * d * hq * pairs                         # the impact pass's own QK^T
+    kv_doc = 2 * sum(lay.doc_lens) * hk * d * eb              # K and V gathered, per request
+    k_doc = kv_doc // 2
+    tq = lay.total_q
+    qkv = tq * (hq + 2 * hk) * d * eb
+    o_bytes = tq * hq * d * eb
+    imp_bytes = (lay.total_doc + tq) * 4
+    per_layer_attn_bytes = kv_doc + qkv + o_bytes
+    impact_bytes = k_doc + tq * (hq + hk) * d * eb + imp_bytes
+    L = w.num_layers
+    return {
+        "attn_flops_per_launch": attn_flops,
+        "attn_bytes_per_launch": per_layer_attn_bytes,
+        "impact_flops_per_launch": impact_flops,
+        "impact_bytes_per_launch": impact_bytes,
+        "step_flops": attn_flops * L,
+        "step_bytes": per_layer_attn_bytes * L + imp_bytes * 2,
+        "doc_tokens": sum(lay.doc_lens),
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_sources_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "serving_prefill_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(config, kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it matches these sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    j = json.load(open(p))
+    e = j.get(f"{config}/{kernel}")
+    if not e or e.get("src_digest") != kernel_sources_digest():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+class Replica:
+    """One independent copy of the step's device inputs and buffers."""
+
+    def __init__(self, w, lay, layer_inputs, device):
+        from serving_prefill_b200 import Batch, KVPool
+        from serving_prefill_b200.engine import PrefillEngine, write_chunks
+        self.pool = KVPool(w.num_layers, lay.num_pages, w.num_kv_heads, w.head_dim, dtype=w.torch_dtype,
+                           device=device)
+        self.batch = Batch(lay.req_chunk_off, lay.chunk_doc_off, lay.chunk_page_off, lay.page_ids, lay.q_off,
+                           device=device)
+        self.engine = PrefillEngine(self.pool, self.batch, w.num_q_heads, w.r, dtype=w.torch_dtype, device=device)
+        pages = [p.to(torch.int32).to(device) for p in lay.chunk_pages]
+        self.layers = []
+        for layer in range(w.num_layers):
+            inp = layer_inputs[layer]
+            write_chunks(self.pool, layer, pages, [k.to(device) for k in inp.chunk_k],
+                         [v.to(device) for v in inp.chunk_v])
+            self.layers.append((layer, inp.q.to(device), inp.kq.to(device), inp.vq.to(device)))
+        tq = lay.total_q
+        self.outs = [torch.empty(max(tq, 1), w.num_q_heads, w.head_dim, dtype=w.torch_dtype, device=device)
+                     for _ in range(w.num_layers)]
+        self.impact_layer = w.impact_layer_index
+        self.graph = None
+
+    def step(self):
+        self.engine.step(self.layers, self.impact_layer, outs=self.outs)
+
+    def capture(self):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.step()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+        torch.cuda.synchronize()
+
+    def nbytes(self):
+        return self.pool.k.numel() * self.pool.k.element_size() * 2 + sum(
+            t.numel() * t.element_size() for _, q, kq, vq in self.layers for t in (q, kq, vq))
+
+
+def run_gpu(args, w, rank, world, device):
+    import serving_prefill_b200 as sp
+    torch.cuda.set_device(device)
+    lay = make_layout(w)
+    layer_inputs = [make_layer_inputs(w, lay, layer) for layer in range(w.num_layers)]
+    work = step_work(w, lay)
+    first = Replica(w, lay, layer_inputs, device)
+    per_copy = first.nbytes()
+    n_copies = max(1, min(16, -(-2 * L2_BYTES // per_copy)))
+    free = torch.cuda.mem_get_info(device)[0]
+    n_copies = max(1, min(n_copies, int(0.5 * free // max(per_copy, 1)) + 1))
+    reps = [first] + [Replica(w, lay, layer_inputs, device) for _ in range(n_copies - 1)]
+    for r in reps:
+        r.step()
+    torch.cuda.synchronize()
+    st, bits = first.engine.device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} bits {bits}")
+    for r in reps:
+        r.capture()
+
+    # warm-up
+    for i in range(args.warmup):
+        reps[i % n_copies].graph.replay()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    clocks = ClockSampler(device if isinstance(device, int) else torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.2)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for i in range(args.steps):
+        reps[i % n_copies].graph.replay()
+    ev1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    # launches inside the timed region: graph replays carry the captured kernels
+    per_step_launches = None
+
+    # per-kernel timing pass (eager launches, events around every kernel)
+    sp.rag_profile_enable(True)
+    base = sp.rag_launch_count()
+    prof_steps = max(3, min(args.steps, 200))
+    for i in range(prof_steps):
+        reps[i % n_copies].step()
+    torch.cuda.synchronize()
+    per_step_launches = (sp.rag_launch_count() - base) / prof_steps
+    prof = sp.rag_profile_collect()
+    sp.rag_profile_enable(False)
+    clk = clocks.stop()
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = world * work["doc_tokens"] * args.steps / (ms_max / 1e3)
+
+    # dominant kernel and its roofline
+    peaks = load_peaks()
+    kinds = {k: v for k, v in prof.items() if v[1] > 0}
+    dom = max(kinds, key=lambda k: kinds[k][0])
+    dom_ms, dom_n = kinds[dom]
+    avg_s = dom_ms / dom_n / 1e3
+    per_launch = {
+        "attn": (work["attn_flops_per_launch"], work["attn_bytes_per_launch"]),
+        "combine": (0, 0),
+        "impact": (work["impact_flops_per_launch"], work["impact_bytes_per_launch"]),
+        "topk": (0, (lay.total_doc + lay.total_q) * 4),
+        "simt_attn": (work["attn_flops_per_launch"], work["attn_bytes_per_launch"]),
+        "simt_impact": (work["impact_flops_per_launch"], work["impact_bytes_per_launch"]),
+    }.get(dom, (0, 0))
+    flops, nbytes = per_launch
+    long_region = ms > 1000.0
+    tflops_peak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
+    ridge = tflops_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops and flops / max(nbytes, 1) > ridge:
+        achieved = flops / avg_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tflops_peak, "unit": "TFLOP/s",
+                "frac": achieved / tflops_peak}
+    else:
+        achieved = nbytes / avg_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    roof["kernel"] = dom
+    roof["peak_source"] = peaks["source"]
+    roof["avg_launch_us"] = avg_s * 1e6
+    roof["traffic"] = recorded_traffic(args.config, dom)
+    t_roof = max(work["step_flops"] / (tflops_peak * 1e12), work["step_bytes"] / (peaks["hbm_gbs"] * 1e9))
+    step_roof = {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step / 1e3)}
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(args, w, lay, layer_inputs, first, device, world)
+
+    kernels = {k: {"ms_per_step": v[0] / prof_steps, "launches_per_step": v[1] / prof_steps} for k, v in kinds.items()}
+    return {
+        "value": value, "ms_per_step": ms_per_step, "roofline": roof, "step_roofline": step_roof,
+        "e2e": e2e, "gpu_launches": int(round(per_step_launches * args.steps)), "clocks": clk,
+        "kernels": kernels, "copies": n_copies, "work": work,
+    }
+
+
+def run_e2e(args, w, lay, layer_inputs, rep, device, world):
+    """Same step through the C ABI with pinned host inputs and outputs."""
+    from serving_prefill_b200 import rag_fused_prefill_attn, rag_impact_topk
+    eng = rep.engine
+    host_in = []
+    for layer in range(w.num_layers):
+        inp = layer_inputs[layer]
+        host_in.append(tuple(t.contiguous().pin_memory() for t in (inp.q, inp.kq, inp.vq)))
+    desc = [t.contiguous().pin_memory() for t in rep.batch.host]
+    dev_in = [(q.to(device), kq.to(device), vq.to(device)) for q, kq, vq in host_in]
+    host_topk = torch.empty_like(eng.topk_idx, device="cpu").pin_memory()
+    host_o = [torch.empty_like(o, device="cpu").pin_memory() for o in rep.outs]
+    h2d = sum(t.numel() * t.element_size() for trip in host_in for t in trip) + sum(
+        t.numel() * t.element_size() for t in desc)
+    d2h = host_topk.numel() * 4 + sum(o.numel() * o.element_size() for o in host_o)
+    steps = max(3, min(args.steps, 50))
+
+    def one():
+        for t, dt in zip(desc, rep.batch.dev):
+            if t.numel():
+                dt[: t.numel()].copy_(t, non_blocking=True)
+        for layer in range(w.num_layers):
+            q, kq, vq = dev_in[layer]
+            hq, hkq, hvq = host_in[layer]
+            q.copy_(hq, non_blocking=True)
+            kq.copy_(hkq, non_blocking=True)
+            vq.copy_(hvq, non_blocking=True)
+            rag_fused_prefill_attn(rep.pool, layer, rep.batch, q, kq, vq, rep.outs[layer], eng.ws,
+                                   impact=eng.impact if layer == w.impact_layer_index else None,
+                                   row_lse=eng.row_lse)
+            host_o[layer].copy_(rep.outs[layer], non_blocking=True)
+        rag_impact_topk(eng.impact, rep.batch, w.r, eng.k_cap, eng.topk_idx, eng.topk_val, eng.k)
+        host_topk.copy_(eng.topk_idx, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(steps):
+        one()
+    ev1.record()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(t.item())
+    doc = sum(lay.doc_lens)
+    return {"value": world * doc * steps / (ms / 1e3), "unit": "doc-KV tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step(w, lay, layer_inputs, heads):
+    """The oracle on a sample of query heads of every layer, then top-k."""
+    import oracle.prefill as orc
+    scale = 1.0 / np.sqrt(w.head_dim)
+    bits = np.uint16 if w.dtype == "bf16" else np.uint32
+    impact_all = None
+    for layer in range(w.num_layers):
+        inp = layer_inputs[layer]
+        pk, pv = orc.build_layer_pool(lay, inp, bits)
+        q_all, kq_all, vq_all = orc.to_f64(inp.q), orc.to_f64(inp.kq), orc.to_f64(inp.vq)
+        G = w.num_q_heads // w.num_kv_heads
+        q0 = 0
+        imps = []
+        for b, cs in enumerate(lay.req_chunks):
+            ql = lay.q_lens[b]
+            chunks = [(lay.chunk_pages[c].numpy(), lay.chunk_len[c]) for c in cs]
+            kd = orc.bits_to_f64(orc.gather(pk, 0, chunks))
+            vd = orc.bits_to_f64(orc.gather(pv, 0, chunks))
+            n_doc = kd.shape[0]
+            kcat = np.concatenate([kd, kq_all[q0:q0 + ql]])
+            vcat = np.concatenate([vd, vq_all[q0:q0 + ql]])
+            sel_q = q_all[q0:q0 + ql][:, heads, :]
+            kv_heads = sorted({h // G for h in heads})
+            remap = [kv_heads.index(h // G) for h in heads]
+            ks = kcat[:, kv_heads, :][:, remap, :]
+            vs = vcat[:, kv_heads, :][:, remap, :]
+            _, _, _, imp, _ = orc.attend_request(sel_q, ks, vs, n_doc, scale,
+                                                 want_impact=(layer == w.impact_layer_index))
+            if imp is not None:
+                k = orc.recompute_count(n_doc, w.r)
+                orc.select_topk(imp[:n_doc], k)
+                imps.append(imp)
+            q0 += ql
+        if imps:
+            impact_all = imps
+    return impact_all
+
+
+def run_reference(args, w, budget_per_step=None):
+    lay = make_layout(w)
+    layer_inputs = [make_layer_inputs(w, lay, layer) for layer in range(w.num_layers)]
+    doc = sum(lay.doc_lens)
+    # calibrate: one head of every layer
+    t0 = time.perf_counter()
+    oracle_step(w, lay, layer_inputs, [0])
+    t_head = max(time.perf_counter() - t0, 1e-3)
+    budget = budget_per_step or max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    n_heads = int(max(1, min(w.num_q_heads, budget // t_head)))
+    heads = list(range(0, w.num_q_heads, max(1, w.num_q_heads // n_heads)))[:n_heads]
+    for _ in range(args.warmup):
+        oracle_step(w, lay, layer_inputs, heads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(w, lay, layer_inputs, heads)
+    dt = time.perf_counter() - t0
+    frac = len(heads) / w.num_q_heads
+    value = doc * frac * args.steps / dt
+    sample = (f"{len(heads)} of {w.num_q_heads} query heads of every layer (gather, attention, impact, "
+              f"top-k over all doc tokens); tokens/s scaled by the head fraction")
+    return value, dt / args.steps, sample
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    w = get_workload(args.config)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        value, s_per_step, sample = run_reference(args, w)
+        cores = blas_threads()
+        line = {
+            "impl": "reference", "metric": METRIC, "value": value, "unit": "doc-KV tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s_per_step * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "requests": len(make_layout(w).q_lens), "layers": w.num_layers},
+            "cpu_baseline": {"value": value, "unit": "doc-KV tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "doc-KV tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    device = local
+    res = run_gpu(args, w, rank, world, device)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        small = argparse.Namespace(steps=2, warmup=1)
+        value, s_per_step, sample = run_reference(small, w, budget_per_step=5.0)
+        cpu = {"value": value, "unit": "doc-KV tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": sample + f"; 2 timed steps of {s_per_step:.2f} s"}
+
+    if rank == 0:
+        lay = make_layout(w)
+        line = {
+            "metric": METRIC, "value": res["value"], "unit": "doc-KV tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "requests": lay.num_requests, "layers": w.num_layers,
+                       "doc_tokens_per_step": sum(lay.doc_lens), "query_tokens_per_step": lay.total_q,
+                       "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                       "r": w.r, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs rotated over {res['copies']} copies (> L2) between steps",
+                       "timing": "CUDA graph replay per step"},
+            "roofline": res["roofline"], "step_roofline": res["step_roofline"],
+            "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
+            "clocks": res["clocks"], "kernels": res["kernels"],
+        }
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -580,8 +580,12 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const CUtensorMap& tkq, const CUtensorMap& tvq, const FwdParams& p, int grid,
                             cudaStream_t stream) {
   const size_t smem = fwd_smem_bytes(p.batch.num_requests);
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
+  static size_t attr_set = 0;   // largest dynamic smem size configured so far
+  if (smem > attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    attr_set = smem;
+  }
   attn_fwd_kernel<<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, tkq, tvq, p);
   return cudaGetLastError();
 }

@@ -150,8 +150,12 @@ cudaError_t launch_topk(const TopkParams& p, int num_requests, int max_k, cudaSt
   int kp = 1;
   while (kp < max_k) kp <<= 1;
   const size_t smem = sizeof(uint64_t) * size_t(kp);
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
+  static size_t attr_set = 0;   // largest dynamic smem size configured so far
+  if (smem > attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    attr_set = smem;
+  }
   topk_kernel<<<num_requests, kTopkThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
