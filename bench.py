@@ -444,6 +444,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu", action="store_true",
+                    help="profiling mode: one input copy, eager launches, W + K steps, no JSON")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     w = get_workload(args.config)
@@ -475,6 +477,16 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     device = local
+    if args.ncu:
+        torch.cuda.set_device(device)
+        lay = make_layout(w)
+        rep = Replica(w, lay, [make_layer_inputs(w, lay, layer) for layer in range(w.num_layers)], device)
+        for _ in range(args.warmup + args.steps):
+            rep.step()
+        torch.cuda.synchronize()
+        st, bits = rep.engine.device_error()
+        print(f"ncu mode: {args.warmup + args.steps} steps of {w.name}, device status {st} ({bits})")
+        sys.exit(0 if st == 0 else 1)
     res = run_gpu(args, w, rank, world, device)
 
     cpu = None

@@ -29,7 +29,7 @@ constexpr int kDescSlots = 4;
 constexpr int kTileBytes = kBN * kHeadDim * 2;   // one K or V tile, bf16
 constexpr int kHalfBytes = kTileBytes / 2;       // 64 columns of d
 constexpr int kQBytes = kBM * kHeadDim * 2;
-constexpr int kFwdThreads = 224;                 // 4 softmax + K + V + MMA warps
+constexpr int kFwdThreads = 256;                 // 4 softmax + K + V + MMA + V-convert warps
 constexpr float kRescaleThreshold = 8.0f;        // log2 units: rescale O when the max grows by > 2^8
 
 // TMEM columns
@@ -45,7 +45,7 @@ struct TileDesc {
 struct FwdCtrl {
   uint64_t q_full, q_empty;
   uint64_t kfull[kKStages], kempty[kKStages];
-  uint64_t vfull[kVStages], vempty[kVStages];
+  uint64_t vfull[kVStages], vempty[kVStages], vconv[kVStages];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t o_free, teardown;
   uint64_t desc_full[kDescSlots], desc_empty[kDescSlots];
@@ -146,7 +146,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(&ctl->q_full, 1);
     mbar_init(&ctl->q_empty, 1);
     for (int s = 0; s < kKStages; ++s) { mbar_init(&ctl->kfull[s], 1); mbar_init(&ctl->kempty[s], 1); }
-    for (int s = 0; s < kVStages; ++s) { mbar_init(&ctl->vfull[s], 1); mbar_init(&ctl->vempty[s], 1); }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&ctl->vfull[s], 1);
+      mbar_init(&ctl->vempty[s], 1);
+      mbar_init(&ctl->vconv[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->s_full[s], 1);
       mbar_init(&ctl->p_full[s], 128);
@@ -307,7 +311,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float a = ex2(x[64 * h + 2 * j] - m_use);
             const float b2 = ex2(x[64 * h + 2 * j + 1] - m_use);
             ls += a + b2;
-            pk[j] = pack_bf16x2(a, b2);
+            pk[j] = pack_f16x2(a, b2);
           }
           tmem_st32(tmem + lane_off + (buf ? kColP1 : kColP0) + 32 * h, pk);
         }
@@ -452,11 +456,43 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (is_k && ctl->abort && q_iter > 0) wait_quiet(&ctl->q_full, (q_iter - 1) & 1);
     }
     __syncwarp();
+  } else if (warp == 7) {
+    // ------------------------------------------------------------ V converter
+    // The PV product runs in fp16 (P and V): P keeps 3 more mantissa bits than
+    // bf16, and every bf16 V value of magnitude in [2^-14, 65504] is exact in
+    // fp16. The tile is rewritten in place; the 128B swizzle is unchanged.
+    uint32_t t_glob = 0;
+    int bad = 0;
+    for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
+      const FwdItem it = decode_fwd_item(p, prefix, w);
+      const int n = it.t_end - it.t_begin;
+      for (int i = 0; i < n; ++i) {
+        const uint32_t t = t_glob + i;
+        const int s = t % kVStages;
+        if (!mbar_wait(&ctl->vfull[s], (t / kVStages) & 1, abort_flag)) { bad = 1; break; }
+        uint4* tile = reinterpret_cast<uint4*>(sV + s * kTileBytes);
+#pragma unroll 4
+        for (int v = lane; v < kTileBytes / 16; v += 32) {
+          uint4 x = tile[v];
+          x.x = bf16x2_to_f16x2(x.x);
+          x.y = bf16x2_to_f16x2(x.y);
+          x.z = bf16x2_to_f16x2(x.z);
+          x.w = bf16x2_to_f16x2(x.w);
+          tile[v] = x;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->vconv[s]);
+      }
+      t_glob += n;
+    }
+    if (bad) raise_abort(ctl, p.err);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0);
-      const uint32_t idesc_pv = idesc_bf16_f32(kBM, kHeadDim, 1);
+      const uint32_t idesc_pv = idesc_f16_f32(kBM, kHeadDim, 1);
       const uint32_t q_base = smem_u32(sQ);
       uint32_t t_glob = 0, q_iter = 0, o_uses = 0;
       int bad = 0;
@@ -488,7 +524,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               ++o_uses;
             }
             if (!mbar_wait(&ctl->p_full[tp & 1], (tp >> 1) & 1, abort_flag)) { bad = 1; break; }
-            if (!mbar_wait(&ctl->vfull[sv], (tp / kVStages) & 1, abort_flag)) { bad = 1; break; }
+            if (!mbar_wait(&ctl->vconv[sv], (tp / kVStages) & 1, abort_flag)) { bad = 1; break; }
             tc_fence_after();
             const uint32_t v_base = smem_u32(sV + sv * kTileBytes);
             const uint32_t a_p = tmem + ((tp & 1) ? kColP1 : kColP0);
@@ -523,54 +559,61 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 // ---------------------------------------------------------------- combine
 
 
-// Merge the split partials (O, m, l) of one (request, kv head, row tile):
-// m = max_s m_s, l = sum_s l_s 2^(m_s - m), O = sum_s O_s 2^(m_s - m) / l.
-// grid: x = kv head * max row tiles + row tile, y = request; 8 warps, warp per row.
+// Merge the split partials (O, m, l) of every row, in one pass:
+//   m = max_s m_s, l = sum_s l_s 2^(m_s - m), O = sum_s O_s 2^(m_s - m) / l.
+// grid: x = (kv head * max row tiles + row tile) * 16 + group of 8 rows,
+// y = request; one warp per row, each lane owns 4 of the 128 columns.
+constexpr int kCombineRowsPerBlock = 8;
+
 __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p, int max_rt) {
+  const int groups = kBM / kCombineRowsPerBlock;
   const int b = blockIdx.y;
-  const int g = blockIdx.x / max_rt;
-  const int rt = blockIdx.x % max_rt;
+  const int unit = blockIdx.x / groups;
+  const int g = unit / max_rt;
+  const int rt = unit % max_rt;
   const ReqInfo req = load_req(p.batch, b);
   const FwdShape sh = fwd_shape(p.batch, req, p.group, p.tiles_per_split);
   if (rt >= sh.n_rt || g >= p.num_kv_heads) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.group;
+  const int r = (blockIdx.x % groups) * kCombineRowsPerBlock + warp;
+  const int pr = rt * kBM + r;
+  const int tok = pr / G;
+  if (tok >= req.n_q) return;
+  const int head = g * G + pr % G;
   const int base = p.item_prefix[b];
-  for (int r = warp; r < kBM; r += 8) {
-    const int pr = rt * kBM + r;
-    const int tok = pr / G;
-    if (tok >= req.n_q) break;
-    const int head = g * G + pr % G;
-    float m = -INFINITY;
-    for (int s = 0; s < sh.n_split; ++s) {
-      const size_t slot = size_t(base) + (size_t(g) * sh.n_split + s) * sh.n_rt + rt;
-      if (slot >= size_t(p.max_items) || size_t(base) >= size_t(p.item_prefix[p.batch.num_requests])) return;
-      m = fmaxf(m, p.part[(slot * kBM + r) * kPartStride + kHeadDim]);
+  const size_t first = size_t(base) + size_t(g) * sh.n_split * sh.n_rt + rt;
+  if (first + size_t(sh.n_split - 1) * sh.n_rt >= size_t(p.max_items)) return;
+  float m = -INFINITY, l = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int s = 0; s < sh.n_split; ++s) {
+    const float* row = p.part + ((first + size_t(s) * sh.n_rt) * kBM + r) * kPartStride;
+    const float2 ml = *reinterpret_cast<const float2*>(row + kHeadDim);
+    const float4 v = reinterpret_cast<const float4*>(row)[lane];
+    if (ml.x == -INFINITY) continue;
+    if (ml.x > m) {
+      const float c = (m == -INFINITY) ? 0.f : ex2(m - ml.x);
+      acc.x = acc.x * c + v.x; acc.y = acc.y * c + v.y; acc.z = acc.z * c + v.z; acc.w = acc.w * c + v.w;
+      l = l * c + ml.y;
+      m = ml.x;
+    } else {
+      const float c = ex2(ml.x - m);
+      acc.x += v.x * c; acc.y += v.y * c; acc.z += v.z * c; acc.w += v.w * c;
+      l += ml.y * c;
     }
-    const float m_use = (m == -INFINITY) ? 0.f : m;
-    float l = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < sh.n_split; ++s) {
-      const size_t slot = size_t(base) + (size_t(g) * sh.n_split + s) * sh.n_rt + rt;
-      const float* pr_row = p.part + (slot * kBM + r) * kPartStride;
-      const float ms = pr_row[kHeadDim];
-      const float ls = pr_row[kHeadDim + 1];
-      const float wgt = (ms == -INFINITY) ? 0.f : ex2(ms - m_use);
-      l += ls * wgt;
-      const float4 v = reinterpret_cast<const float4*>(pr_row)[lane];
-      acc.x += v.x * wgt; acc.y += v.y * wgt; acc.z += v.z * wgt; acc.w += v.w * wgt;
-    }
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    const int64_t row = int64_t(req.q0 + tok) * p.num_q_heads + head;
-    uint2 out;
-    out.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    out.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    reinterpret_cast<uint2*>(p.o + row * kHeadDim)[lane] = out;
-    if (lane == 0) {
-      p.row_m2[row] = m_use;
-      p.row_il[row] = l > 0.f ? 1.f / (l * float(p.num_q_heads)) : 0.f;
-      if (p.row_lse) p.row_lse[row] = (m_use + __log2f(l)) * 0.69314718055994531f;
-    }
+  }
+  const float m_use = (m == -INFINITY) ? 0.f : m;
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  const int64_t orow = int64_t(req.q0 + tok) * p.num_q_heads + head;
+  uint2 out;
+  out.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  out.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  reinterpret_cast<uint2*>(p.o + orow * kHeadDim)[lane] = out;
+  if (lane == 0) {
+    p.row_m2[orow] = m_use;
+    p.row_il[orow] = l > 0.f ? 1.f / (l * float(p.num_q_heads)) : 0.f;
+    if (p.row_lse) p.row_lse[orow] = (m_use + __log2f(l)) * 0.69314718055994531f;
   }
 }
 
@@ -591,7 +634,7 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
 }
 
 cudaError_t launch_attn_combine(const CombineParams& p, int max_rt, int num_requests, cudaStream_t stream) {
-  dim3 grid(p.num_kv_heads * max_rt, num_requests);
+  dim3 grid(p.num_kv_heads * max_rt * (kBM / kCombineRowsPerBlock), num_requests);
   attn_combine_kernel<<<grid, 256, 0, stream>>>(p, max_rt);
   return cudaGetLastError();
 }

@@ -462,6 +462,8 @@ rag_status rag_impact_topk(const float* impact, const rag_batch* batch, double r
   p.r = r;
   p.k_cap = k_cap;
   p.k_max = std::max(kmax, 1);
+  // full sort when every request fits the 64 KB sort buffer, else radix select
+  p.sort_cap = b.max_doc <= 8192 ? std::max(b.max_doc, 1) : 0;
   p.topk_idx = topk_idx;
   p.topk_val = topk_val;
   p.k_out = k_out;
