@@ -166,6 +166,30 @@ RAG_API rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer
                                   float* row_lse, float* impact, void* workspace, size_t workspace_bytes,
                                   void* stream);
 
+/* Same computation as rag_fused_prefill_attn, for callers that cannot
+ * allocate device memory (a runtime that gives a plugin only its input and
+ * output buffers, a deployment whose device memory is planned once at start-up,
+ * a loop that must never wait on an allocator). The pages have no counterpart
+ * of this entry point; it exists only for such callers.
+ * Instead of a caller workspace it uses one fixed device array of 64 MiB that
+ * lives in this library's device image: every GPU on which the library has been
+ * loaded keeps it until the process exits, and nothing is allocated per call.
+ * A batch whose workspace (rag_workspace_size) exceeds 64 MiB is rejected with
+ * RAG_ERR_WORKSPACE before anything is launched.
+ * All calls share that one array and it keeps the last call's contents: the
+ * call clears the error word it needs zeroed, but calls that overlap on the GPU
+ * (different streams, or different host threads, on one device) race on it;
+ * serialise them on one stream.
+ * The first call on each device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.
+ * device_err: optional device int32 that receives the call's device error bits
+ * (as rag_last_device_error reports them: 1 page, 2 geometry, 4 timeout).
+ * Other arguments and outputs as for rag_fused_prefill_attn. */
+RAG_API rag_status rag_fused_prefill_attn_static(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch,
+                                                 const void* q, int32_t num_q_heads, const void* kq,
+                                                 const void* vq, float sm_scale, void* o, float* row_lse,
+                                                 float* impact, int32_t* device_err, void* stream);
+
 /* Recompute count for a request with n_doc doc tokens (CacheBlend page,
  * "Recompute ratio trade-off" and listing): max(1, int(n_doc * r)) with the
  * product in double precision, and 0 when n_doc is 0. Host function. */

@@ -58,6 +58,9 @@ EXPORTS = {
     "rag_fused_prefill_attn": (c_int32, [POINTER(RagKVPool), c_int32, POINTER(RagBatch), c_void_p, c_int32,
                                          c_void_p, c_void_p, c_float, c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_size_t, c_void_p]),
+    "rag_fused_prefill_attn_static": (c_int32, [POINTER(RagKVPool), c_int32, POINTER(RagBatch), c_void_p,
+                                                c_int32, c_void_p, c_void_p, c_float, c_void_p, c_void_p,
+                                                c_void_p, c_void_p, c_void_p]),
     "rag_recompute_count": (c_int32, [c_int32, c_double]),
     "rag_impact_topk": (c_int32, [c_void_p, POINTER(RagBatch), c_double, c_int32, c_void_p, c_void_p, c_void_p,
                                   c_void_p]),
@@ -193,6 +196,19 @@ def rag_fused_prefill_attn(pool: KVPool, layer: int, batch: Batch, q: torch.Tens
                                         _ptr(kq), _ptr(vq), sm_scale, _ptr(o), _ptr(row_lse), _ptr(impact),
                                         _ptr(workspace), workspace.numel(), _stream(stream)),
            "rag_fused_prefill_attn")
+
+
+def rag_fused_prefill_attn_static(pool: KVPool, layer: int, batch: Batch, q: torch.Tensor, kq: torch.Tensor,
+                                  vq: torch.Tensor, o: torch.Tensor, impact: torch.Tensor = None,
+                                  row_lse: torch.Tensor = None, device_err: torch.Tensor = None,
+                                  sm_scale: float = 0.0, stream=None):
+    """rag_fused_prefill_attn without a workspace: for callers that cannot
+    allocate device memory; scratch is the library's fixed 64 MiB device array."""
+    num_q_heads = q.shape[1] if q.dim() == 3 else 0
+    _check(lib().rag_fused_prefill_attn_static(ctypes.byref(pool.c), layer, ctypes.byref(batch.c), _ptr(q),
+                                               num_q_heads, _ptr(kq), _ptr(vq), sm_scale, _ptr(o), _ptr(row_lse),
+                                               _ptr(impact), _ptr(device_err), _stream(stream)),
+           "rag_fused_prefill_attn_static")
 
 
 def rag_impact_topk(impact: torch.Tensor, batch: Batch, r: float, k_cap: int, topk_idx: torch.Tensor,
