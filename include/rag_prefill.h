@@ -227,6 +227,11 @@ RAG_API int64_t rag_launch_count(void);
 RAG_API void rag_profile_enable(int32_t on);
 RAG_API rag_status rag_profile_collect(double* ms, int64_t* launches, int32_t n_kinds);
 
+/* Like rag_profile_collect, but keeps the record. Launches recorded while a
+ * stream was being captured into a CUDA graph become event nodes of the graph;
+ * after each replay this reads that replay's per-kernel device times. */
+RAG_API rag_status rag_profile_peek(double* ms, int64_t* launches, int32_t n_kinds);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,6 +20,7 @@ from .rag import (  # noqa: F401
     rag_launch_count,
     rag_num_sms,
     rag_profile_collect,
+    rag_profile_peek,
     rag_profile_enable,
     rag_recompute_count,
     rag_workspace_size,

@@ -3,18 +3,25 @@
 // (TurboRAG page, "Technical Details": Concat of the per-chunk caches and the
 // query's own K/V; causal attention softmax(QK^T/sqrt(d_k) + M_causal) V).
 //
-// One persistent CTA per SM walks work items (request, kv head, 128-row tile,
-// split of the key tiles). Rows pack the G query heads of one KV head with
-// the query tokens (row = token * G + head-in-group), so GQA groups share
-// every K/V tile in the MMA M dimension. Per 128-key tile:
-//   K producer warp : page table -> 8 TMA page boxes (or one box of K_q)
+// One persistent CTA per SM walks work items (request, kv head, 256-row
+// block, split of the key tiles). Rows pack the G query heads of one KV head
+// with the query tokens (row = token * G + head-in-group), so GQA groups share
+// every K/V tile in the MMA M dimension. A block is two 128-row Q tiles that
+// share each 128-key K/V tile:
+//   K producer warp : Q tiles, then page table -> 8 TMA page boxes per K tile
+//                     (or one box of K_q), and the tile's mask descriptor
 //   V producer warp : the same for V
-//   MMA warp        : S = Q K^T (tcgen05, smem x smem -> TMEM), then
-//                     O += P V (tcgen05, P from TMEM x V from smem)
-//   4 softmax warps : thread = row = TMEM lane; mask, online max/sum in the
-//                     log2 domain, P (bf16) back to TMEM, lazy O rescale
-// S and P are double-buffered in TMEM so QK^T of tile t+1 overlaps the
-// softmax of tile t. Every wait is bounded; a timeout raises a device error.
+//   V converter warp: V tile bf16 -> fp16 in place (PV runs in fp16)
+//   MMA warp        : S_i = Q_i K^T (tcgen05 smem x smem -> TMEM) for both Q
+//                     tiles, then O_i += P_i V (P_i from TMEM, V from smem)
+//   2 x 4 softmax warps: warpgroup i owns Q tile i; thread = row = TMEM lane;
+//                     mask, online max/sum in the log2 domain, P_i (fp16)
+//                     written over the columns of S_i, lazy O_i rescale
+// The two softmax warpgroups alternate with the tensor core: while one
+// computes exponentials the MMA warp runs the other Q tile's products.
+// A fixed share of the exponentials runs as a polynomial on the FMA pipe to
+// relieve the MUFU unit. Every wait is bounded; a timeout raises a device
+// error instead of hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -23,31 +30,32 @@
 
 namespace rag {
 
-constexpr int kKStages = 3;
+constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr int kDescSlots = 4;
-constexpr int kTileBytes = kBN * kHeadDim * 2;   // one K or V tile, bf16
+constexpr int kTileBytes = kBN * kHeadDim * 2;   // one K, V or Q tile, 16-bit
 constexpr int kHalfBytes = kTileBytes / 2;       // 64 columns of d
-constexpr int kQBytes = kBM * kHeadDim * 2;
-constexpr int kFwdThreads = 256;                 // 4 softmax + K + V + MMA + V-convert warps
+constexpr int kFwdThreads = 384;                 // 8 softmax + K + V + MMA + convert warps
 constexpr float kRescaleThreshold = 8.0f;        // log2 units: rescale O when the max grows by > 2^8
+constexpr int kPolyPairsOf8 = 3;                 // of every 8 column pairs, 3 use the FMA-pipe exp2
 
-// TMEM columns
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+// TMEM columns: S_i (P_i aliased over its first 64 columns), O_i
+__host__ __device__ constexpr uint32_t col_s(int qt) { return 128u * qt; }
+__host__ __device__ constexpr uint32_t col_o(int qt) { return 256u + 128u * qt; }
 
 struct TileDesc {
   int32_t kind;       // 0: doc tile from the pool, 1: query-key tile
   int32_t kbase;      // query tile: index of its first query key
+  int32_t full;       // doc tile: every slot of the 8 pages is a real token
   uint8_t nvalid[kPagesPerTile];
 };
-
 
 struct FwdCtrl {
   uint64_t q_full, q_empty;
   uint64_t kfull[kKStages], kempty[kKStages];
   uint64_t vfull[kVStages], vempty[kVStages], vconv[kVStages];
-  uint64_t s_full[2], p_full[2], pv_done[2];
-  uint64_t o_free, teardown;
+  uint64_t s_full[kQTiles], p_full[kQTiles], pv_done[kQTiles], o_free[kQTiles];
+  uint64_t teardown;
   uint64_t desc_full[kDescSlots], desc_empty[kDescSlots];
   TileDesc desc[kDescSlots];
   uint32_t tmem_base;
@@ -55,14 +63,15 @@ struct FwdCtrl {
   int32_t total_items;
 };
 
-constexpr size_t kFwdSmemData = kQBytes + size_t(kKStages + kVStages) * kTileBytes;
+constexpr size_t kFwdSmemData = size_t(kQTiles + kKStages + kVStages) * kTileBytes;
 
 __host__ size_t fwd_smem_bytes(int num_requests) {
   return 1024 + kFwdSmemData + sizeof(FwdCtrl) + sizeof(int32_t) * (num_requests + 1) + 64;
 }
 
 struct FwdItem {
-  int b, g, rt, split;
+  int b, g, rb, split;
+  int n_qt;             // active Q tiles (1 or 2)
   int t_begin, t_end;   // tiles of the unit handled by this item
   int n_doc_tiles;
   ReqInfo req;
@@ -80,12 +89,14 @@ __device__ __forceinline__ FwdItem decode_fwd_item(const FwdParams& p, const int
   it.req = load_req(p.batch, lo);
   const FwdShape sh = fwd_shape(p.batch, it.req, p.group, p.tiles_per_split);
   int local = w - prefix[lo];
-  it.rt = local % sh.n_rt;
+  it.rb = local % sh.n_rt;
   local /= sh.n_rt;
   it.split = local % sh.n_split;
   it.g = local / sh.n_split;
+  const int rows = it.req.n_q * p.group - it.rb * kFwdRows;
+  it.n_qt = rows > kBM ? 2 : 1;
   it.n_doc_tiles = doc_tiles(it.req);
-  const int last_tok = min(it.req.n_q, (it.rt + 1) * kBM / p.group) - 1;
+  const int last_tok = min(it.req.n_q, (it.rb + 1) * kFwdRows / p.group) - 1;
   const int n_tiles = it.n_doc_tiles + query_tiles_upto(last_tok);
   it.t_begin = min(it.split * p.tiles_per_split, n_tiles);
   it.t_end = min(it.t_begin + p.tiles_per_split, n_tiles);
@@ -105,8 +116,8 @@ __device__ __forceinline__ void wait_quiet(uint64_t* bar, uint32_t parity) {
   mbar_wait(bar, parity, &zero);
 }
 
-// K-major, 128B-swizzled tile of 128 rows x 128 bf16 stored as two 64-column
-// halves of 16 KB; k-step kk covers columns [16 kk, 16 kk + 16).
+// K-major, 128B-swizzled tile of 128 rows x 128 16-bit values stored as two
+// 64-column halves of 16 KB; k-step kk covers columns [16 kk, 16 kk + 16).
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk) {
   return sdesc_sw128(base + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
 }
@@ -117,6 +128,22 @@ __device__ __forceinline__ uint64_t v_desc(uint32_t base, int kk) {
   return sdesc_sw128(base + kk * 16 * 128, kHalfBytes, 1024);
 }
 
+// 2^x on the FMA pipe: x = n + f with n = round(x), f in [-1/2, 1/2];
+// 2^f by a degree-3 polynomial (minimax for relative error on [-1/2, 1/2],
+// fitted for this library with the Remez exchange; max relative error 7.5e-5),
+// 2^n by adding n to the exponent field. Inputs below -126 are clamped (their
+// result, ~1e-38, is below every fp16/fp32 sum it enters).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float magic = 12582912.0f;            // 1.5 * 2^23: x + magic rounds x to an integer
+  const float t = x + magic;
+  const float f = x - (t - magic);
+  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kq,
@@ -124,7 +151,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + kQBytes;
+  uint8_t* sK = sQ + kQTiles * kTileBytes;
   uint8_t* sV = sK + kKStages * kTileBytes;
   FwdCtrl* ctl = reinterpret_cast<FwdCtrl*>(sV + kVStages * kTileBytes);
   int32_t* prefix = reinterpret_cast<int32_t*>(ctl + 1);
@@ -151,25 +178,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(&ctl->vempty[s], 1);
       mbar_init(&ctl->vconv[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&ctl->s_full[s], 1);
-      mbar_init(&ctl->p_full[s], 128);
-      mbar_init(&ctl->pv_done[s], 1);
+    for (int q = 0; q < kQTiles; ++q) {
+      mbar_init(&ctl->s_full[q], 1);
+      mbar_init(&ctl->p_full[q], 128);
+      mbar_init(&ctl->pv_done[q], 1);
+      mbar_init(&ctl->o_free[q], 128);
     }
-    mbar_init(&ctl->o_free, 128);
     mbar_init(&ctl->teardown, 1);
-    for (int s = 0; s < kDescSlots; ++s) { mbar_init(&ctl->desc_full[s], 1); mbar_init(&ctl->desc_empty[s], 4); }
+    for (int s = 0; s < kDescSlots; ++s) {
+      mbar_init(&ctl->desc_full[s], 1);
+      mbar_init(&ctl->desc_empty[s], 8);   // one arrival per softmax warp
+    }
     ctl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 6) {
+  if (warp == 10) {
     tmem_alloc(&ctl->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_kq);
   }
-  if (warp == 5 && lane == 0) { tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_vq); }
+  if (warp == 9 && lane == 0) { tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_vq); }
 
   // per-request item counts -> exclusive prefix (warp 0), total in ctl
   if (warp == 0) {
@@ -214,63 +244,74 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tmem = ctl->tmem_base;
   volatile int* abort_flag = &ctl->abort;
 
-  if (warp < 4) {
-    // ------------------------------------------------------------ softmax
-    const int r = tid;
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
-    uint32_t t_glob = 0;
+  // registers: the softmax warpgroups take 208 per thread, the four role warps 88
+  if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+    // ------------------------------------------------------------ softmax warpgroup qt
+    const int qt = warp >> 2;
+    const int r = tid & 127;
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + col_s(qt);
+    const uint32_t o_addr = tmem + lane_off + col_o(qt);
+    uint32_t t_glob = 0, n_s = 0;   // tiles seen by the CTA, S tiles processed on this Q tile
     int bad = 0;
     for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
       const FwdItem it = decode_fwd_item(p, prefix, w);
       const int n = it.t_end - it.t_begin;
-      const int pr = it.rt * kBM + r;
+      const bool active = qt < it.n_qt;
+      const int pr = it.rb * kFwdRows + qt * kBM + r;
       const int tok = pr / G;
       const int head = it.g * G + (pr % G);
-      const bool row_valid = tok < it.req.n_q;
+      const bool row_valid = active && tok < it.req.n_q;
       float m_ref = -INFINITY, l_sum = 0.f;
       for (int i = 0; i < n; ++i) {
         const uint32_t t = t_glob + i;
-        const uint32_t buf = t & 1;
         const uint32_t slot = t % kDescSlots;
         if (!mbar_wait(&ctl->desc_full[slot], (t / kDescSlots) & 1, abort_flag)) { bad = 1; break; }
         const TileDesc td = ctl->desc[slot];
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->desc_empty[slot]);
-        if (!mbar_wait(&ctl->s_full[buf], (t >> 1) & 1, abort_flag)) { bad = 1; break; }
+        if (!active) continue;
+        if (!mbar_wait(&ctl->s_full[qt], n_s & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
         float x[kBN];
         {
-          uint32_t u[32];
+          uint32_t u0[32], u1[32];
+          tmem_ld32(s_addr + 0, u0);
+          tmem_ld32(s_addr + 32, u1);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            tmem_ld32(tmem + lane_off + (buf ? kColS1 : kColS0) + 32 * c, u);
-            tmem_wait_ld();
+          for (int j = 0; j < 32; ++j) { x[j] = __uint_as_float(u0[j]); x[32 + j] = __uint_as_float(u1[j]); }
+          tmem_ld32(s_addr + 64, u0);
+          tmem_ld32(s_addr + 96, u1);
+          tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) x[32 * c + j] = __uint_as_float(u[j]);
-          }
+          for (int j = 0; j < 32; ++j) { x[64 + j] = __uint_as_float(u0[j]); x[96 + j] = __uint_as_float(u1[j]); }
         }
-        // mask and move to the log2 domain
-        float mx = -INFINITY;
+        // mask (only partial tiles), then the row max of the raw scores
         if (td.kind == 0) {
-          uint32_t nv_lo = *reinterpret_cast<const uint32_t*>(&td.nvalid[0]);
-          uint32_t nv_hi = *reinterpret_cast<const uint32_t*>(&td.nvalid[4]);
+          if (!td.full) {
+            const uint32_t nv_lo = *reinterpret_cast<const uint32_t*>(&td.nvalid[0]);
+            const uint32_t nv_hi = *reinterpret_cast<const uint32_t*>(&td.nvalid[4]);
 #pragma unroll
-          for (int c = 0; c < kBN; ++c) {
-            const int pg = c >> 4;
-            const uint32_t nv = ((pg < 4 ? nv_lo >> (8 * pg) : nv_hi >> (8 * (pg - 4))) & 0xffu);
-            const float v = (uint32_t(c & 15) < nv) ? x[c] * p.scale_log2 : -INFINITY;
-            x[c] = v;
-            mx = fmaxf(mx, v);
+            for (int c = 0; c < kBN; ++c) {
+              const int pg = c >> 4;
+              const uint32_t nv = ((pg < 4 ? nv_lo >> (8 * pg) : nv_hi >> (8 * (pg - 4))) & 0xffu);
+              if (uint32_t(c & 15) >= nv) x[c] = -INFINITY;
+            }
           }
         } else {
           const int lim = tok - td.kbase;   // keys c <= lim are visible
+          if (lim < kBN - 1) {
 #pragma unroll
-          for (int c = 0; c < kBN; ++c) {
-            const float v = (c <= lim) ? x[c] * p.scale_log2 : -INFINITY;
-            x[c] = v;
-            mx = fmaxf(mx, v);
+            for (int c = 0; c < kBN; ++c)
+              if (c > lim) x[c] = -INFINITY;
           }
         }
+        float mx = x[0];
+#pragma unroll
+        for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, x[c]);
+        mx = mx * p.scale_log2;   // scale > 0: max of scaled = scaled max
         float alpha = 1.f;
         bool need = false;
         if (i == 0) {
@@ -280,65 +321,68 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           need = true;
         }
         if (__any_sync(0xffffffffu, need)) {
-          // O must hold PV of the previous tile before it is rescaled
-          const uint32_t tp = t - 1;
-          if (!mbar_wait(&ctl->pv_done[tp & 1], (tp >> 1) & 1, abort_flag)) { bad = 1; break; }
+          // O must hold the previous tile's PV before it is rescaled
+          if (!mbar_wait(&ctl->pv_done[qt], (n_s - 1) & 1, abort_flag)) { bad = 1; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t u[32];
-            tmem_ld32(tmem + lane_off + kColO + 32 * c, u);
+            tmem_ld32(o_addr + 32 * c, u);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * alpha);
-            tmem_st32(tmem + lane_off + kColO + 32 * c, u);
+            tmem_st32(o_addr + 32 * c, u);
           }
           tmem_wait_st();
           if (need) { l_sum *= alpha; m_ref = mx; }
         }
-        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // P buffer `buf` was last read by PV of tile t - 2
-        if (t >= 2) {
-          const uint32_t tq = t - 2;
-          if (!mbar_wait(&ctl->pv_done[buf], (tq >> 1) & 1, abort_flag)) { bad = 1; break; }
-        }
+        const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
         float ls = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float a = ex2(x[64 * h + 2 * j] - m_use);
-            const float b2 = ex2(x[64 * h + 2 * j + 1] - m_use);
+            const float ya = fmaf(x[64 * h + 2 * j], p.scale_log2, neg_m);
+            const float yb = fmaf(x[64 * h + 2 * j + 1], p.scale_log2, neg_m);
+            float a, b2;
+            if ((j & 7) < kPolyPairsOf8) {
+              a = exp2_poly(ya);
+              b2 = exp2_poly(yb);
+            } else {
+              a = ex2(ya);
+              b2 = ex2(yb);
+            }
             ls += a + b2;
             pk[j] = pack_f16x2(a, b2);
           }
-          tmem_st32(tmem + lane_off + (buf ? kColP1 : kColP0) + 32 * h, pk);
+          tmem_st32(s_addr + 32 * h, pk);   // P over the first 64 columns of S
         }
         l_sum += ls;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&ctl->p_full[buf]);
+        mbar_arrive(&ctl->p_full[qt]);
+        ++n_s;
       }
       if (bad) break;
       t_glob += n;
+      if (!active) continue;
 
-      // ---- epilogue: O of this item
+      // ---- epilogue: O of this Q tile
       float o[kHeadDim];
       if (n > 0) {
-        const uint32_t tl = t_glob - 1;
-        if (!mbar_wait(&ctl->pv_done[tl & 1], (tl >> 1) & 1, abort_flag)) { bad = 1; break; }
+        if (!mbar_wait(&ctl->pv_done[qt], (n_s - 1) & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t u[32];
-          tmem_ld32(tmem + lane_off + kColO + 32 * c, u);
+          tmem_ld32(o_addr + 32 * c, u);
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[32 * c + j] = __uint_as_float(u[j]);
         }
         tc_fence_before();
-        mbar_arrive(&ctl->o_free);
+        mbar_arrive(&ctl->o_free[qt]);
       } else {
 #pragma unroll
         for (int j = 0; j < kHeadDim; ++j) o[j] = 0.f;
@@ -363,16 +407,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (p.row_lse) p.row_lse[row] = (m_use + __log2f(l_sum)) * 0.69314718055994531f;
         }
       } else {
-        float4* dst = reinterpret_cast<float4*>(p.part + (size_t(w) * kBM + r) * kPartStride);
+        float4* dst = reinterpret_cast<float4*>(p.part + ((size_t(w) * kQTiles + qt) * kBM + r) * kPartStride);
 #pragma unroll
         for (int c = 0; c < kHeadDim / 4; ++c) dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
         dst[kHeadDim / 4] = make_float4(m_ref, l_sum, 0.f, 0.f);
       }
     }
     if (bad) raise_abort(ctl, p.err);
-  } else if (warp == 4 || warp == 5) {
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+    if (warp == 8 || warp == 9) {
     // ------------------------------------------------------------ producers
-    const bool is_k = (warp == 4);
+    const bool is_k = (warp == 8);
     const CUtensorMap* tm_pool = is_k ? &tm_k : &tm_v;
     const CUtensorMap* tm_qkv = is_k ? &tm_kq : &tm_vq;
     uint8_t* sbase = is_k ? sK : sV;
@@ -388,10 +434,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (is_k) {
         if (q_iter > 0 && !mbar_wait(&ctl->q_empty, (q_iter - 1) & 1, abort_flag)) { bad = 1; break; }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&ctl->q_full, kQBytes);
-          const int tok0 = it.req.q0 + it.rt * (kBM / G);
-          tma_load_3d(sQ, &tm_q, &ctl->q_full, 0, it.g * G, tok0);
-          tma_load_3d(sQ + kHalfBytes, &tm_q, &ctl->q_full, 64, it.g * G, tok0);
+          mbar_arrive_expect_tx(&ctl->q_full, it.n_qt * kTileBytes);
+          for (int q = 0; q < it.n_qt; ++q) {
+            const int tok0 = it.req.q0 + (it.rb * kFwdRows + q * kBM) / G;
+            tma_load_3d(sQ + q * kTileBytes, &tm_q, &ctl->q_full, 0, it.g * G, tok0);
+            tma_load_3d(sQ + q * kTileBytes + kHalfBytes, &tm_q, &ctl->q_full, 64, it.g * G, tok0);
+          }
         }
         ++q_iter;
       }
@@ -410,12 +458,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             break;
           }
           TileDesc* d = &ctl->desc[slot];
+          const unsigned full_pages = __ballot_sync(0xffffffffu, lane < kPagesPerTile && pg.nvalid == kPage);
           if (doc) {
             if (lane < kPagesPerTile) d->nvalid[lane] = uint8_t(pg.nvalid);
-            if (lane == 0) { d->kind = 0; d->kbase = 0; }
+            if (lane == 0) { d->kind = 0; d->kbase = 0; d->full = (full_pages == 0xffu) ? 1 : 0; }
           } else if (lane == 0) {
             d->kind = 1;
             d->kbase = (tile - it.n_doc_tiles) * kBN;
+            d->full = 0;
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl->desc_full[slot]);
@@ -444,19 +494,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       t_glob += n;
     }
-    if (bad) {
-      raise_abort(ctl, p.err);
-    }
+    if (bad) raise_abort(ctl, p.err);
     // let every copy this warp issued land before the CTA exits
-    if (lane == 0) {
-      const uint32_t issued = t_glob;
-      const uint32_t first = issued > uint32_t(nstages) ? issued - nstages : 0;
-      if (ctl->abort)
-        for (uint32_t t = first; t < issued; ++t) wait_quiet(&full[t % nstages], (t / nstages) & 1);
-      if (is_k && ctl->abort && q_iter > 0) wait_quiet(&ctl->q_full, (q_iter - 1) & 1);
+    if (lane == 0 && ctl->abort) {
+      const uint32_t first = t_glob > uint32_t(nstages) ? t_glob - nstages : 0;
+      for (uint32_t t = first; t < t_glob; ++t) wait_quiet(&full[t % nstages], (t / nstages) & 1);
+      if (is_k && q_iter > 0) wait_quiet(&ctl->q_full, (q_iter - 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 7) {
+  } else if (warp == 11) {
     // ------------------------------------------------------------ V converter
     // The PV product runs in fp16 (P and V): P keeps 3 more mantissa bits than
     // bf16, and every bf16 V value of magnitude in [2^-14, 65504] is exact in
@@ -489,12 +535,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (bad) raise_abort(ctl, p.err);
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ MMA issuer (warp 10)
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0);
       const uint32_t idesc_pv = idesc_f16_f32(kBM, kHeadDim, 1);
       const uint32_t q_base = smem_u32(sQ);
-      uint32_t t_glob = 0, q_iter = 0, o_uses = 0;
+      uint32_t t_glob = 0, q_iter = 0;
+      uint32_t n_pv[kQTiles] = {0, 0}, n_item[kQTiles] = {0, 0};   // PVs issued, items begun, per Q tile
       int bad = 0;
       for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
         const FwdItem it = decode_fwd_item(p, prefix, w);
@@ -502,38 +549,56 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (n == 0) continue;
         if (!mbar_wait(&ctl->q_full, q_iter & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
+        // Tensor-core order per step: PV_0(t-1), QK_0(t), PV_1(t-1), QK_1(t), so
+        // that softmax 0 of tile t runs while the pipe does PV_1 and QK_1.
         for (int i = 0; i <= n && !bad; ++i) {
-          if (i < n) {
-            const uint32_t t = t_glob + i;
-            const int s = t % kKStages;
-            if (!mbar_wait(&ctl->kfull[s], (t / kKStages) & 1, abort_flag)) { bad = 1; break; }
-            tc_fence_after();
-            const uint32_t k_base = smem_u32(sK + s * kTileBytes);
-            const uint32_t d_s = tmem + ((t & 1) ? kColS1 : kColS0);
-#pragma unroll
-            for (int kk = 0; kk < kHeadDim / 16; ++kk)
-              mma_ss(d_s, kmajor_desc(q_base, kk), kmajor_desc(k_base, kk), idesc_qk, kk > 0);
-            tc_commit(&ctl->s_full[t & 1]);
-            tc_commit(&ctl->kempty[s]);
-          }
+          const uint32_t t = t_glob + i;          // tile of the QK products of this step
+          const uint32_t tp = t - 1;              // tile of the PV products of this step
+          const int s = t % kKStages;
+          const int sv = tp % kVStages;
+          uint32_t v_base = 0, k_base = 0;
           if (i >= 1) {
-            const uint32_t tp = t_glob + i - 1;
-            const int sv = tp % kVStages;
-            if (i == 1) {
-              if (o_uses > 0 && !mbar_wait(&ctl->o_free, (o_uses - 1) & 1, abort_flag)) { bad = 1; break; }
-              ++o_uses;
-            }
-            if (!mbar_wait(&ctl->p_full[tp & 1], (tp >> 1) & 1, abort_flag)) { bad = 1; break; }
             if (!mbar_wait(&ctl->vconv[sv], (tp / kVStages) & 1, abort_flag)) { bad = 1; break; }
-            tc_fence_after();
-            const uint32_t v_base = smem_u32(sV + sv * kTileBytes);
-            const uint32_t a_p = tmem + ((tp & 1) ? kColP1 : kColP0);
-#pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
-              mma_ts(tmem + kColO, a_p + kk * 8, v_desc(v_base, kk), idesc_pv, (i > 1) || (kk > 0));
-            tc_commit(&ctl->pv_done[tp & 1]);
-            tc_commit(&ctl->vempty[sv]);
+            v_base = smem_u32(sV + sv * kTileBytes);
           }
+          if (i < n) {
+            if (!mbar_wait(&ctl->kfull[s], (t / kKStages) & 1, abort_flag)) { bad = 1; break; }
+            k_base = smem_u32(sK + s * kTileBytes);
+          }
+          for (int q = 0; q < it.n_qt && !bad; ++q) {
+            if (i >= 1) {
+              // O_q += P_q V for the previous tile
+              if (i == 1) {
+                if (n_item[q] > 0 && !mbar_wait(&ctl->o_free[q], (n_item[q] - 1) & 1, abort_flag)) {
+                  bad = 1;
+                  break;
+                }
+                ++n_item[q];
+              }
+              if (!mbar_wait(&ctl->p_full[q], n_pv[q] & 1, abort_flag)) { bad = 1; break; }
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < kBN / 16; ++kk)
+                mma_ts(tmem + col_o(q), tmem + col_s(q) + kk * 8, v_desc(v_base, kk), idesc_pv,
+                       (i > 1) || (kk > 0));
+              tc_commit(&ctl->pv_done[q]);
+              ++n_pv[q];
+            }
+            if (i < n) {
+              // S_q = Q_q K^T for this tile. It overwrites P_q (aliased over S_q),
+              // which PV_q of the previous tile reads: tcgen05.mma operations of
+              // one CTA execute in issue order, so no completion wait is needed.
+              tc_fence_after();
+              const uint32_t qb = q_base + q * kTileBytes;
+#pragma unroll
+              for (int kk = 0; kk < kHeadDim / 16; ++kk)
+                mma_ss(tmem + col_s(q), kmajor_desc(qb, kk), kmajor_desc(k_base, kk), idesc_qk, kk > 0);
+              tc_commit(&ctl->s_full[q]);
+            }
+          }
+          if (bad) break;
+          if (i >= 1) tc_commit(&ctl->vempty[sv]);
+          if (i < n) tc_commit(&ctl->kempty[s]);
         }
         if (bad) break;
         tc_commit(&ctl->q_empty);
@@ -546,11 +611,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       wait_quiet(&ctl->teardown, 0);
     }
     __syncwarp();
+    }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 6) {
+  if (warp == 10) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -558,37 +624,36 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
 // ---------------------------------------------------------------- combine
 
-
 // Merge the split partials (O, m, l) of every row, in one pass:
 //   m = max_s m_s, l = sum_s l_s 2^(m_s - m), O = sum_s O_s 2^(m_s - m) / l.
-// grid: x = (kv head * max row tiles + row tile) * 16 + group of 8 rows,
+// grid: x = (kv head * max row blocks + row block) * 32 + group of 8 rows,
 // y = request; one warp per row, each lane owns 4 of the 128 columns.
 constexpr int kCombineRowsPerBlock = 8;
 
-__global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p, int max_rt) {
-  const int groups = kBM / kCombineRowsPerBlock;
+__global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p, int max_rb) {
+  const int groups = kFwdRows / kCombineRowsPerBlock;
   const int b = blockIdx.y;
   const int unit = blockIdx.x / groups;
-  const int g = unit / max_rt;
-  const int rt = unit % max_rt;
+  const int g = unit / max_rb;
+  const int rb = unit % max_rb;
   const ReqInfo req = load_req(p.batch, b);
   const FwdShape sh = fwd_shape(p.batch, req, p.group, p.tiles_per_split);
-  if (rt >= sh.n_rt || g >= p.num_kv_heads) return;
+  if (rb >= sh.n_rt || g >= p.num_kv_heads) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.group;
-  const int r = (blockIdx.x % groups) * kCombineRowsPerBlock + warp;
-  const int pr = rt * kBM + r;
+  const int rr = (blockIdx.x % groups) * kCombineRowsPerBlock + warp;   // row within the 256-row block
+  const int pr = rb * kFwdRows + rr;
   const int tok = pr / G;
   if (tok >= req.n_q) return;
   const int head = g * G + pr % G;
   const int base = p.item_prefix[b];
-  const size_t first = size_t(base) + size_t(g) * sh.n_split * sh.n_rt + rt;
+  const size_t first = size_t(base) + size_t(g) * sh.n_split * sh.n_rt + rb;
   if (first + size_t(sh.n_split - 1) * sh.n_rt >= size_t(p.max_items)) return;
   float m = -INFINITY, l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
   for (int s = 0; s < sh.n_split; ++s) {
-    const float* row = p.part + ((first + size_t(s) * sh.n_rt) * kBM + r) * kPartStride;
+    const float* row = p.part + ((first + size_t(s) * sh.n_rt) * kFwdRows + rr) * kPartStride;
     const float2 ml = *reinterpret_cast<const float2*>(row + kHeadDim);
     const float4 v = reinterpret_cast<const float4*>(row)[lane];
     if (ml.x == -INFINITY) continue;
@@ -633,9 +698,9 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_combine(const CombineParams& p, int max_rt, int num_requests, cudaStream_t stream) {
-  dim3 grid(p.num_kv_heads * max_rt * (kBM / kCombineRowsPerBlock), num_requests);
-  attn_combine_kernel<<<grid, 256, 0, stream>>>(p, max_rt);
+cudaError_t launch_attn_combine(const CombineParams& p, int max_rb, int num_requests, cudaStream_t stream) {
+  dim3 grid(p.num_kv_heads * max_rb * (kFwdRows / kCombineRowsPerBlock), num_requests);
+  attn_combine_kernel<<<grid, 256, 0, stream>>>(p, max_rb);
   return cudaGetLastError();
 }
 

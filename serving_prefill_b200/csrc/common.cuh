@@ -11,7 +11,9 @@ namespace rag {
 
 constexpr int kPage = 16;             // tokens per pool page
 constexpr int kHeadDim = 128;         // head_dim of the tensor-core path
-constexpr int kBM = 128;              // attention rows (query token x head-in-group) per tile
+constexpr int kBM = 128;              // attention rows (query token x head-in-group) per Q tile
+constexpr int kQTiles = 2;            // Q tiles per attention work item
+constexpr int kFwdRows = kBM * kQTiles;
 constexpr int kBN = 128;              // keys per tile
 constexpr int kPagesPerTile = kBN / kPage;
 constexpr int kImpactRows = 256;      // rows per impact-pass block (MMA N)
@@ -71,14 +73,14 @@ __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b -
 // the query block's keys in tiles of 128.
 __device__ __forceinline__ int doc_tiles(const ReqInfo& r) { return ceil_div(r.n_pages, kPagesPerTile); }
 
-// Attention work units: (request, kv head, 128-row tile, split of the key tiles).
+// Attention work units: (request, kv head, 256-row block, split of the key tiles).
 struct FwdShape {
   int n_rt, n_split;
 };
 __device__ __forceinline__ FwdShape fwd_shape(const BatchDev& B, const ReqInfo& r, int G, int tiles_per_split) {
   FwdShape s;
   if (r.n_q <= 0 || !req_ok(B, r)) { s.n_rt = 0; s.n_split = 0; return s; }
-  s.n_rt = ceil_div(r.n_q * G, kBM);
+  s.n_rt = ceil_div(r.n_q * G, kFwdRows);
   s.n_split = ceil_div(doc_tiles(r) + ceil_div(r.n_q, kBN), tiles_per_split);
   return s;
 }
@@ -150,7 +152,7 @@ __device__ __forceinline__ PageRef page_ref(const BatchDev& B, const ReqInfo& r,
 //   item prefix                (kMaxRequests + 1) int32
 //   row_m2                     total_q * H_q fp32   (reference max, log2 units)
 //   row_il                     total_q * H_q fp32   (1 / (l * H_q))
-//   partials                   items * 128 * kPartStride fp32
+//   partials                   items * 256 * kPartStride fp32
 struct WsLayout {
   size_t off_prefix, off_m2, off_il, off_part, total;
 };
@@ -163,7 +165,7 @@ __host__ __device__ inline WsLayout ws_layout(int64_t total_q, int num_q_heads, 
   w.off_prefix = at; at = align256(at + sizeof(int32_t) * (kMaxRequests + 1));
   w.off_m2 = at; at = align256(at + sizeof(float) * size_t(total_q) * num_q_heads);
   w.off_il = at; at = align256(at + sizeof(float) * size_t(total_q) * num_q_heads);
-  w.off_part = at; at = align256(at + sizeof(float) * size_t(max_items) * kBM * kPartStride);
+  w.off_part = at; at = align256(at + sizeof(float) * size_t(max_items) * kFwdRows * kPartStride);
   w.total = at;
   return w;
 }

@@ -53,7 +53,6 @@ struct TopkParams {
   double r;
   int32_t k_cap;
   int32_t k_max;           // k of the longest request
-  int32_t sort_cap;        // requests with at most this many doc tokens are fully sorted
   int32_t* topk_idx;
   float* topk_val;
   int32_t* k_out;

@@ -203,7 +203,7 @@ static BatchDev to_dev(const rag_batch& b) {
 
 static size_t workspace_bytes_for(const rag_kv_pool& pool, const rag_batch& b, int num_q_heads) {
   const int G = num_q_heads / pool.num_kv_heads;
-  const Plan pf = plan_split(b, pool.num_kv_heads, G, kBM, num_sms());
+  const Plan pf = plan_split(b, pool.num_kv_heads, G, kFwdRows, num_sms());
   return ws_layout(b.total_q, num_q_heads, pool.dtype == RAG_BF16 ? pf.max_items : 0).total;
 }
 
@@ -350,7 +350,7 @@ rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const 
   // ---- bf16 tensor-core path
   if (kBM % G != 0) return RAG_ERR_UNSUPPORTED;
   const int sms = num_sms();
-  const Plan pf = plan_split(b, pool->num_kv_heads, G, kBM, sms);
+  const Plan pf = plan_split(b, pool->num_kv_heads, G, kFwdRows, sms);
   const WsLayout wl = ws_layout(b.total_q, num_q_heads, pf.max_items);
   const int H_kv = pool->num_kv_heads;
   const uint64_t pool_rows = uint64_t(pool->num_layers) * pool->num_pages * H_kv * kPage;
@@ -462,8 +462,6 @@ rag_status rag_impact_topk(const float* impact, const rag_batch* batch, double r
   p.r = r;
   p.k_cap = k_cap;
   p.k_max = std::max(kmax, 1);
-  // full sort when every request fits the 64 KB sort buffer, else radix select
-  p.sort_cap = b.max_doc <= 8192 ? std::max(b.max_doc, 1) : 0;
   p.topk_idx = topk_idx;
   p.topk_val = topk_val;
   p.k_out = k_out;
@@ -492,6 +490,29 @@ rag_status rag_last_device_error(void* workspace, int32_t* bits, void* stream) {
 int64_t rag_launch_count(void) { return g_launches.load(); }
 
 void rag_profile_enable(int32_t on) { g_prof_on.store(on ? 1 : 0); }
+
+rag_status rag_profile_peek(double* ms, int64_t* launches, int32_t n_kinds) {
+  std::vector<ProfRecord> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    recs = g_prof;
+  }
+  std::vector<double> acc(kNumKinds, 0.0);
+  std::vector<int64_t> cnt(kNumKinds, 0);
+  rag_status st = RAG_OK;
+  for (auto& r : recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+      st = RAG_ERR_CUDA;
+    acc[r.kind] += t;
+    cnt[r.kind] += 1;
+  }
+  for (int i = 0; i < n_kinds && i < kNumKinds; ++i) {
+    if (ms) ms[i] = acc[i];
+    if (launches) launches[i] = cnt[i];
+  }
+  return st;
+}
 
 rag_status rag_profile_collect(double* ms, int64_t* launches, int32_t n_kinds) {
   std::vector<ProfRecord> recs;

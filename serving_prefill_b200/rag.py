@@ -68,6 +68,7 @@ EXPORTS = {
     "rag_launch_count": (c_int64, []),
     "rag_profile_enable": (None, [c_int32]),
     "rag_profile_collect": (c_int32, [c_void_p, c_void_p, c_int32]),
+    "rag_profile_peek": (c_int32, [c_void_p, c_void_p, c_int32]),
 }
 
 
@@ -229,6 +230,14 @@ def rag_launch_count() -> int:
 
 def rag_profile_enable(on: bool):
     lib().rag_profile_enable(1 if on else 0)
+
+
+def rag_profile_peek() -> dict:
+    n = len(KERNEL_KINDS)
+    ms = (c_double * n)()
+    cnt = (c_int64 * n)()
+    _check(lib().rag_profile_peek(ctypes.cast(ms, c_void_p), ctypes.cast(cnt, c_void_p), n), "rag_profile_peek")
+    return {k: (ms[i], cnt[i]) for i, k in enumerate(KERNEL_KINDS)}
 
 
 def rag_profile_collect() -> dict:

@@ -1,0 +1,67 @@
+"""The top-k kernel alone, through the C ABI, on seeded impact vectors.
+
+It is a pure function of the impact vector, so it is checked bit-exactly
+against the oracle's stable sort on the same fp32 values: the whole-sort path
+(short requests), the bucket-candidate path (long requests) and the exact
+fallback when one bucket holds more candidates than fit in shared memory
+(mass ties, all-zero impacts).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.prefill as orc
+from serving_prefill_b200 import Batch, rag_impact_topk, rag_recompute_count
+
+pytestmark = pytest.mark.gpu
+
+
+def run_topk(segments, r):
+    n = [len(s) for s in segments]
+    pages = [-(-x // 16) for x in n]
+    batch = Batch(req_chunk_off=list(range(len(n) + 1)), chunk_doc_off=np.cumsum([0] + n).tolist(),
+                  chunk_page_off=np.cumsum([0] + pages).tolist(), page_ids=list(range(sum(pages))),
+                  q_off=[0] * (len(n) + 1))
+    impact = torch.from_numpy(np.concatenate(segments).astype(np.float32)).cuda()
+    k_cap = max(1, max(rag_recompute_count(x, r) for x in n))
+    idx = torch.empty(len(n), k_cap, dtype=torch.int32, device="cuda")
+    val = torch.empty(len(n), k_cap, dtype=torch.float32, device="cuda")
+    kk = torch.empty(len(n), dtype=torch.int32, device="cuda")
+    rag_impact_topk(impact, batch, r, k_cap, idx, val, kk)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), val.cpu().numpy(), kk.cpu().numpy()
+
+
+def check(segments, r):
+    idx, val, kk = run_topk(segments, r)
+    for b, seg in enumerate(segments):
+        seg32 = seg.astype(np.float32)
+        k = orc.recompute_count(len(seg), r) if len(seg) else 0
+        assert kk[b] == k
+        want = orc.select_topk(seg32.astype(np.float64), k)
+        assert idx[b, :k].tolist() == want.tolist(), f"request {b} (n={len(seg)})"
+        np.testing.assert_array_equal(val[b, :k], seg32[want])
+        assert np.all(idx[b, k:] == -1)
+
+
+def test_short_requests_whole_sort():
+    rng = np.random.default_rng(1)
+    check([rng.random(n) for n in (1, 5, 120, 2048, 8192)], 0.1)
+
+
+def test_long_request_bucket_path():
+    rng = np.random.default_rng(2)
+    check([rng.lognormal(-6, 1.0, 65536), rng.random(20000), rng.lognormal(0, 0.01, 9000)], 0.05)
+
+
+def test_mass_ties_fall_back_to_exact_select():
+    rng = np.random.default_rng(3)
+    few_values = rng.integers(0, 4, 60000).astype(np.float64) / 3.0   # 4 distinct values, ~15k each
+    check([few_values, np.zeros(65536), np.full(10000, 0.25)], 0.1)
+
+
+def test_k_one_and_large_ratio():
+    rng = np.random.default_rng(4)
+    check([rng.random(15), rng.random(9)], 0.1)          # k = 1
+    check([rng.random(12000)], 0.6)                       # k = 7200
