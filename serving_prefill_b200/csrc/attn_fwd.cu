@@ -19,9 +19,10 @@
 //                     written over the columns of S_i, lazy O_i rescale
 // The two softmax warpgroups alternate with the tensor core: while one
 // computes exponentials the MMA warp runs the other Q tile's products.
-// A fixed share of the exponentials runs as a polynomial on the FMA pipe to
-// relieve the MUFU unit. Every wait is bounded; a timeout raises a device
-// error instead of hanging.
+// kPolyPairsOf8 can move a share of the exponentials onto the FMA pipe
+// (exp2_poly2); measured on B200 this pass runs fastest with all of them on
+// MUFU. Every wait is bounded; a timeout raises a device error instead of
+// hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -37,7 +38,7 @@ constexpr int kTileBytes = kBN * kHeadDim * 2;   // one K, V or Q tile, 16-bit
 constexpr int kHalfBytes = kTileBytes / 2;       // 64 columns of d
 constexpr int kFwdThreads = 384;                 // 8 softmax + K + V + MMA + convert warps
 constexpr float kRescaleThreshold = 8.0f;        // log2 units: rescale O when the max grows by > 2^8
-constexpr int kPolyPairsOf8 = 3;                 // of every 8 column pairs, 3 use the FMA-pipe exp2
+constexpr int kPolyPairsOf8 = 0;                 // of every 8 column pairs, this many use the FMA-pipe exp2
 
 // TMEM columns: S_i (P_i aliased over its first 64 columns), O_i
 __host__ __device__ constexpr uint32_t col_s(int qt) { return 128u * qt; }
@@ -58,6 +59,7 @@ struct FwdCtrl {
   uint64_t teardown;
   uint64_t desc_full[kDescSlots], desc_empty[kDescSlots];
   TileDesc desc[kDescSlots];
+  ChunkCache chunks[2];                 // one per producer warp
   uint32_t tmem_base;
   int32_t abort;
   int32_t total_items;
@@ -126,22 +128,6 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk) {
 // 16 KB apart (leading byte offset), 8-key groups 1 KB apart (stride).
 __device__ __forceinline__ uint64_t v_desc(uint32_t base, int kk) {
   return sdesc_sw128(base + kk * 16 * 128, kHalfBytes, 1024);
-}
-
-// 2^x on the FMA pipe: x = n + f with n = round(x), f in [-1/2, 1/2];
-// 2^f by a degree-3 polynomial (minimax for relative error on [-1/2, 1/2],
-// fitted for this library with the Remez exchange; max relative error 7.5e-5),
-// 2^n by adding n to the exponent field. Inputs below -126 are clamped (their
-// result, ~1e-38, is below every fp16/fp32 sum it enters).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float magic = 12582912.0f;            // 1.5 * 2^23: x + magic rounds x to an integer
-  const float t = x + magic;
-  const float f = x - (t - magic);
-  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999280571937561f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -308,9 +294,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               if (c > lim) x[c] = -INFINITY;
           }
         }
-        float mx = x[0];
+        // row max: four independent 3-input max chains
+        float mq[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-        for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, x[c]);
+        for (int c = 4; c < kBN; c += 8) {
+#pragma unroll
+          for (int a = 0; a < 4; ++a) mq[a] = fmax3(mq[a], x[c + 2 * a], x[c + 2 * a + 1]);
+        }
+        float mx = fmax3(fmaxf(mq[0], mq[1]), mq[2], mq[3]);
         mx = mx * p.scale_log2;   // scale > 0: max of scaled = scaled max
         float alpha = 1.f;
         bool need = false;
@@ -337,28 +328,29 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (need) { l_sum *= alpha; m_ref = mx; }
         }
         const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        float ls = 0.f;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(neg_m, neg_m);
+        float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float ya = fmaf(x[64 * h + 2 * j], p.scale_log2, neg_m);
-            const float yb = fmaf(x[64 * h + 2 * j + 1], p.scale_log2, neg_m);
-            float a, b2;
+            const float2 y = ffma2(make_float2(x[64 * h + 2 * j], x[64 * h + 2 * j + 1]), sc2, nm2);
+            float2 e;
             if ((j & 7) < kPolyPairsOf8) {
-              a = exp2_poly(ya);
-              b2 = exp2_poly(yb);
+              e = exp2_poly2(y);
             } else {
-              a = ex2(ya);
-              b2 = ex2(yb);
+              e = make_float2(ex2(y.x), ex2(y.y));
             }
-            ls += a + b2;
-            pk[j] = pack_f16x2(a, b2);
+            ls[j & 3] = fadd2(ls[j & 3], e);
+            pk[j] = pack_f16x2(e.x, e.y);
           }
           tmem_st32(s_addr + 32 * h, pk);   // P over the first 64 columns of S
         }
-        l_sum += ls;
+        const float2 ls01 = fadd2(ls[0], ls[1]), ls23 = fadd2(ls[2], ls[3]);
+        l_sum += (ls01.x + ls01.y) + (ls23.x + ls23.y);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ctl->p_full[qt]);
@@ -431,6 +423,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const FwdItem it = decode_fwd_item(p, prefix, w);
       const int n = it.t_end - it.t_begin;
       if (n == 0) continue;
+      ChunkCache* cc = &ctl->chunks[is_k ? 0 : 1];
+      load_chunk_cache(cc, p.batch, it.req, lane);
+      int32_t next_page = (it.t_begin < it.n_doc_tiles && lane < kPagesPerTile)
+                              ? load_page_id(p.batch, it.req, it.t_begin * kPagesPerTile + lane)
+                              : -1;
       if (is_k) {
         if (q_iter > 0 && !mbar_wait(&ctl->q_empty, (q_iter - 1) & 1, abort_flag)) { bad = 1; break; }
         if (lane == 0) {
@@ -440,6 +437,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_load_3d(sQ + q * kTileBytes, &tm_q, &ctl->q_full, 0, it.g * G, tok0);
             tma_load_3d(sQ + q * kTileBytes + kHalfBytes, &tm_q, &ctl->q_full, 64, it.g * G, tok0);
           }
+          // warm L2 with the Q rows of this CTA's next item
+          const int wn = w + int(gridDim.x);
+          if (wn < total_items) {
+            const FwdItem nx = decode_fwd_item(p, prefix, wn);
+            for (int q = 0; q < nx.n_qt; ++q) {
+              const int tok0 = nx.req.q0 + (nx.rb * kFwdRows + q * kBM) / G;
+              tma_prefetch_3d(&tm_q, 0, nx.g * G, tok0);
+              tma_prefetch_3d(&tm_q, 64, nx.g * G, tok0);
+            }
+          }
         }
         ++q_iter;
       }
@@ -447,10 +454,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t t = t_glob + i;
         const int tile = it.t_begin + i;
         const bool doc = tile < it.n_doc_tiles;
+        const int32_t page_id = next_page;
+        next_page = (tile + 1 < it.n_doc_tiles && lane < kPagesPerTile)
+                        ? load_page_id(p.batch, it.req, (tile + 1) * kPagesPerTile + lane)
+                        : -1;
         PageRef pg;
         pg.page = -1; pg.nvalid = 0; pg.lstart = 0;
         if (doc && lane < kPagesPerTile)
-          pg = page_ref(p.batch, it.req, tile * kPagesPerTile + lane, p.num_pages, is_k ? p.err : nullptr);
+          pg = page_ref_cached(cc, p.batch, it.req, tile * kPagesPerTile + lane, page_id, p.num_pages,
+                               is_k ? p.err : nullptr);
         if (is_k) {
           const uint32_t slot = t % kDescSlots;
           if (t >= kDescSlots && !mbar_wait(&ctl->desc_empty[slot], ((t / kDescSlots) - 1) & 1, abort_flag)) {
@@ -599,9 +611,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (bad) break;
           if (i >= 1) tc_commit(&ctl->vempty[sv]);
           if (i < n) tc_commit(&ctl->kempty[s]);
+          // the drain step reads no Q: the next item's Q may load now
+          if (i == n - 1) tc_commit(&ctl->q_empty);
         }
         if (bad) break;
-        tc_commit(&ctl->q_empty);
         t_glob += n;
         ++q_iter;
       }
@@ -624,7 +637,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
 // ---------------------------------------------------------------- combine
 
-// Merge the split partials (O, m, l) of every row, in one pass:
+// Merge the split partials (O, m, l) of every row:
 //   m = max_s m_s, l = sum_s l_s 2^(m_s - m), O = sum_s O_s 2^(m_s - m) / l.
 // grid: x = (kv head * max row blocks + row block) * 32 + group of 8 rows,
 // y = request; one warp per row, each lane owns 4 of the 128 columns.
@@ -649,26 +662,42 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p
   const int base = p.item_prefix[b];
   const size_t first = size_t(base) + size_t(g) * sh.n_split * sh.n_rt + rb;
   if (first + size_t(sh.n_split - 1) * sh.n_rt >= size_t(p.max_items)) return;
-  float m = -INFINITY, l = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int s = 0; s < sh.n_split; ++s) {
-    const float* row = p.part + ((first + size_t(s) * sh.n_rt) * kFwdRows + rr) * kPartStride;
-    const float2 ml = *reinterpret_cast<const float2*>(row + kHeadDim);
-    const float4 v = reinterpret_cast<const float4*>(row)[lane];
-    if (ml.x == -INFINITY) continue;
-    if (ml.x > m) {
-      const float c = (m == -INFINITY) ? 0.f : ex2(m - ml.x);
-      acc.x = acc.x * c + v.x; acc.y = acc.y * c + v.y; acc.z = acc.z * c + v.z; acc.w = acc.w * c + v.w;
-      l = l * c + ml.y;
-      m = ml.x;
-    } else {
-      const float c = ex2(ml.x - m);
-      acc.x += v.x * c; acc.y += v.y * c; acc.z += v.z * c; acc.w += v.w * c;
-      l += ml.y * c;
-    }
+  // statistics of every split first (lane s holds split s, 32 at a time), then
+  // the weighted rows with several loads in flight
+  const float* row0 = p.part + (first * kFwdRows + rr) * kPartStride;
+  const size_t split_stride = size_t(sh.n_rt) * kFwdRows * kPartStride;
+  float m = -INFINITY;
+  for (int s0 = 0; s0 < sh.n_split; s0 += 32) {
+    const int s = s0 + lane;
+    const float ms = s < sh.n_split ? __ldcg(row0 + s * split_stride + kHeadDim) : -INFINITY;
+    float mm = ms;
+    for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
+    m = fmaxf(m, mm);
   }
   const float m_use = (m == -INFINITY) ? 0.f : m;
+  float l = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < sh.n_split; s0 += 8) {
+    float4 v[8];
+    float2 ml[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (s0 + j < sh.n_split) {
+        const float* row = row0 + (s0 + j) * split_stride;
+        ml[j] = __ldcg(reinterpret_cast<const float2*>(row + kHeadDim));
+        v[j] = __ldcg(reinterpret_cast<const float4*>(row) + lane);
+      } else {
+        ml[j] = make_float2(-INFINITY, 0.f);
+        v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float wgt = (ml[j].x == -INFINITY) ? 0.f : ex2(ml[j].x - m_use);
+      l += ml[j].y * wgt;
+      acc.x += v[j].x * wgt; acc.y += v[j].y * wgt; acc.z += v[j].z * wgt; acc.w += v[j].w * wgt;
+    }
+  }
   const float inv = l > 0.f ? 1.f / l : 0.f;
   const int64_t orow = int64_t(req.q0 + tok) * p.num_q_heads + head;
   uint2 out;

@@ -147,6 +147,69 @@ __device__ __forceinline__ PageRef page_ref(const BatchDev& B, const ReqInfo& r,
   return p;
 }
 
+// A request's chunk table staged in shared memory by a producer warp, so that
+// resolving the 8 pages of a tile costs one global load (the page ids, one
+// tile ahead) instead of a chain of dependent loads.
+constexpr int kChunkCache = 64;
+struct ChunkCache {
+  int32_t n;                            // chunks cached; -1: too many, use global memory
+  int32_t page_off[kChunkCache + 1];    // chunk_page_off[c0 ..= c1]
+  int32_t doc_off[kChunkCache + 1];     // chunk_doc_off[c0 ..= c1]
+};
+
+__device__ __forceinline__ void load_chunk_cache(ChunkCache* cc, const BatchDev& B, const ReqInfo& r, int lane) {
+  const int nc = r.c1 - r.c0;
+  if (nc <= kChunkCache) {
+    for (int i = lane; i <= nc; i += 32) {
+      cc->page_off[i] = __ldg(B.chunk_page_off + r.c0 + i);
+      cc->doc_off[i] = __ldg(B.chunk_doc_off + r.c0 + i);
+    }
+  }
+  if (lane == 0) cc->n = nc <= kChunkCache ? nc : -1;
+  __syncwarp();
+}
+
+// Physical page id of page `ref` of the request (or -1 past its pages).
+__device__ __forceinline__ int32_t load_page_id(const BatchDev& B, const ReqInfo& r, int ref) {
+  return ref < r.n_pages ? __ldg(B.page_ids + r.p0 + ref) : -1;
+}
+
+// page_ref with the chunk table from the cache and a page id loaded earlier.
+__device__ __forceinline__ PageRef page_ref_cached(const ChunkCache* cc, const BatchDev& B, const ReqInfo& r,
+                                                   int ref, int32_t page, int num_pages, int32_t* err) {
+  if (cc->n < 0) return page_ref(B, r, ref, num_pages, err);
+  PageRef p;
+  p.page = -1; p.nvalid = 0; p.lstart = 0;
+  if (ref >= r.n_pages) return p;
+  const int gref = r.p0 + ref;
+  int lo = 0, hi = cc->n - 1;   // last local chunk with page_off <= gref
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cc->page_off[mid] <= gref) lo = mid; else hi = mid - 1;
+  }
+  const int cp0 = cc->page_off[lo], cp1 = cc->page_off[lo + 1];
+  const int k = gref - cp0;
+  const int cstart = cc->doc_off[lo];
+  const int len = cc->doc_off[lo + 1] - cstart;
+  if (k < 0 || gref >= cp1 || len < 0 || cstart < r.doc0 || cstart + len > r.doc0 + r.n_doc) {
+    if (err) atomicOr(err, kDevErrGeometry);
+    return p;
+  }
+  int nv = len - k * kPage;
+  if (nv <= 0 || (gref == cp1 - 1 && nv > kPage)) {
+    if (err) atomicOr(err, kDevErrGeometry);
+  }
+  nv = nv < 0 ? 0 : (nv > kPage ? kPage : nv);
+  if (page < 0 || page >= num_pages) {
+    if (err) atomicOr(err, kDevErrPage);
+    return p;
+  }
+  p.page = page;
+  p.nvalid = nv;
+  p.lstart = cstart - r.doc0 + k * kPage;
+  return p;
+}
+
 // Workspace layout (bytes, each region 256-aligned):
 //   [0, 256)                   error word and flags
 //   item prefix                (kMaxRequests + 1) int32

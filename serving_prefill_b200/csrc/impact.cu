@@ -29,7 +29,8 @@ constexpr int kITileBytes = kBN * kHeadDim * 2;     // K tile
 constexpr int kIHalf = kITileBytes / 2;
 constexpr int kIQHalf = kImpactRows * 128;          // 256 rows x 64 d (bf16) per d-half
 constexpr int kIQBytes = 2 * kIQHalf;
-constexpr int kImpThreads = 192;
+constexpr int kImpThreads = 320;              // 8 epilogue + producer + MMA warps
+constexpr int kImpPolyPairsOf8 = 3;          // of every 8 column pairs, 3 use the FMA-pipe exp2
 
 struct ImpDesc {
   int32_t kind;      // 0 doc tile, 1 query-key tile
@@ -46,7 +47,10 @@ struct ImpCtrl {
   uint64_t teardown;
   uint64_t desc_full[kIDescSlots], desc_empty[kIDescSlots];
   ImpDesc desc[kIDescSlots];
-  float2 mi[kImpactRows];
+  ChunkCache chunks;
+  alignas(16) float neg_m2[kImpactRows];   // -m of every row of the block (log2 units; -inf: no row)
+  alignas(16) float il[kImpactRows];       // 1 / (l * H_q) of every row
+  float red[2][kBN];                      // second-half column sums, per S buffer
   uint32_t tmem_base;
   int32_t abort;
   int32_t total_items;
@@ -85,7 +89,7 @@ __device__ __forceinline__ ImpItem decode_imp_item(const ImpactParams& p, const 
   it.t_begin = min(it.split * p.tiles_per_split, n_tiles);
   it.t_end = min(it.t_begin + p.tiles_per_split, n_tiles);
   it.nrows = min(kImpactRows, it.req.n_q * G - it.rb * kImpactRows);
-  it.N = (it.nrows + 31) & ~31;
+  it.N = (it.nrows + 63) & ~63;   // two halves of whole 32-column TMEM loads
   return it;
 }
 
@@ -121,17 +125,17 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     mbar_init(&ctl->q_full, 1);
     mbar_init(&ctl->q_empty, 1);
     for (int s = 0; s < kIKStages; ++s) { mbar_init(&ctl->kfull[s], 1); mbar_init(&ctl->kempty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&ctl->s_full[s], 1); mbar_init(&ctl->s_free[s], 128); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&ctl->s_full[s], 1); mbar_init(&ctl->s_free[s], 256); }
     mbar_init(&ctl->teardown, 1);
-    for (int s = 0; s < kIDescSlots; ++s) { mbar_init(&ctl->desc_full[s], 1); mbar_init(&ctl->desc_empty[s], 4); }
+    for (int s = 0; s < kIDescSlots; ++s) { mbar_init(&ctl->desc_full[s], 1); mbar_init(&ctl->desc_empty[s], 8); }
     ctl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&ctl->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) { tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_kq); }
+  if (warp == 8 && lane == 0) { tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_kq); }
   if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < B; base += 32) {
@@ -161,28 +165,37 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const uint32_t tmem = ctl->tmem_base;
   volatile int* abort_flag = &ctl->abort;
 
-  if (warp < 4) {
+  if (warp < 8) {
     // ------------------------------------------------------------ epilogue: thread = key
-    const int k = tid;
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    // Two warps per TMEM lane quarter: warp w and w + 4 share 32 keys and take
+    // one half of the block's rows each; the halves meet in shared memory.
+    const int half = warp >> 2;
+    const int k = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     uint32_t t_glob = 0;
     int bad = 0;
     for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
       const ImpItem it = decode_imp_item(p, prefix, w);
       const int n = it.t_end - it.t_begin;
       if (n == 0) continue;
-      named_bar_sync(1, 128);
-      for (int r = tid; r < kImpactRows; r += 128) {
-        float2 v = make_float2(INFINITY, 0.f);
+      named_bar_sync(1, 256);
+      {
+        const int r = tid;   // 256 epilogue threads, one row each
+        float nm = -INFINITY, iv = 0.f;
         if (r < it.nrows) {
           const int pr = it.rb * kImpactRows + r;
           const int64_t row = int64_t(it.req.q0 + pr / G) * p.num_q_heads + it.g * G + pr % G;
-          v = make_float2(p.row_m2[row], p.row_il[row]);
+          nm = -p.row_m2[row];
+          iv = p.row_il[row];
         }
-        ctl->mi[r] = v;
+        ctl->neg_m2[r] = nm;
+        ctl->il[r] = iv;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, 256);
       float* seg = p.impact + (it.req.doc0 + it.req.q0);
+      const int cols = it.N >> 1;         // rows of this half (multiple of 16)
+      const int c0 = half * cols;
       for (int i = 0; i < n; ++i) {
         const uint32_t t = t_glob + i;
         const uint32_t buf = t & 1;
@@ -206,35 +219,56 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (lane == 0) mbar_arrive(&ctl->desc_empty[slot]);
         if (!mbar_wait(&ctl->s_full[buf], (t >> 1) & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
-        float acc = 0.f;
-        const uint32_t col = tmem + lane_off + (buf ? 256u : 0u);
-        for (int c = 0; c < it.N; c += 32) {
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        const uint32_t col = tmem + lane_off + (buf ? 256u : 0u) + c0;
+        for (int c = 0; c < cols; c += 32) {
           uint32_t u[32];
           tmem_ld32(col + c, u);
           tmem_wait_ld();
-          if (kind == 0) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float2 mi = ctl->mi[c + j];
-              acc += ex2(__uint_as_float(u[j]) * p.scale_log2 - mi.x) * mi.y;
+          for (int j = 0; j < 32; j += 4) {
+            const int r0 = c0 + c + j;
+            const float4 nm = *reinterpret_cast<const float4*>(&ctl->neg_m2[r0]);
+            const float4 iv = *reinterpret_cast<const float4*>(&ctl->il[r0]);
+            const float2 x01 = ffma2(make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1])), sc2,
+                                     make_float2(nm.x, nm.y));
+            const float2 x23 = ffma2(make_float2(__uint_as_float(u[j + 2]), __uint_as_float(u[j + 3])), sc2,
+                                     make_float2(nm.z, nm.w));
+            float2 e01, e23;
+            if (((j >> 1) & 7) < kImpPolyPairsOf8) {
+              e01 = exp2_poly2(x01);
+            } else {
+              e01 = make_float2(ex2(x01.x), ex2(x01.y));
             }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float2 mi = ctl->mi[c + j];
-              const float pv = ex2(__uint_as_float(u[j]) * p.scale_log2 - mi.x) * mi.y;
-              acc += (c + j >= rlim) ? pv : 0.f;
+            if ((((j >> 1) + 1) & 7) < kImpPolyPairsOf8) {
+              e23 = exp2_poly2(x23);
+            } else {
+              e23 = make_float2(ex2(x23.x), ex2(x23.y));
             }
+            if (kind != 0) {
+              if (r0 < rlim) e01.x = 0.f;
+              if (r0 + 1 < rlim) e01.y = 0.f;
+              if (r0 + 2 < rlim) e23.x = 0.f;
+              if (r0 + 3 < rlim) e23.y = 0.f;
+            }
+            acc0 = ffma2(e01, make_float2(iv.x, iv.y), acc0);
+            acc1 = ffma2(e23, make_float2(iv.z, iv.w), acc1);
           }
         }
         tc_fence_before();
         mbar_arrive(&ctl->s_free[buf]);
-        if (valid) atomicAdd(seg + lpos, acc);
+        float total = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+        if (half == 1) ctl->red[buf][k] = total;
+        named_bar_sync(2, 256);
+        if (half == 0) {
+          total += ctl->red[buf][k];
+          if (valid) atomicAdd(seg + lpos, total);
+        }
       }
       t_glob += n;
     }
     if (bad) imp_abort(ctl, p.err);
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     // ------------------------------------------------------------ producer
     uint32_t t_glob = 0, q_iter = 0;
     int bad = 0;
@@ -242,6 +276,10 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const ImpItem it = decode_imp_item(p, prefix, w);
       const int n = it.t_end - it.t_begin;
       if (n == 0) continue;
+      load_chunk_cache(&ctl->chunks, p.batch, it.req, lane);
+      int32_t next_page = (it.t_begin < it.n_doc_tiles && lane < kPagesPerTile)
+                              ? load_page_id(p.batch, it.req, it.t_begin * kPagesPerTile + lane)
+                              : -1;
       if (q_iter > 0 && !mbar_wait(&ctl->q_empty, (q_iter - 1) & 1, abort_flag)) { bad = 1; break; }
       if (lane == 0) {
         const int nbox = (it.N + kBM - 1) / kBM;
@@ -257,10 +295,15 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t t = t_glob + i;
         const int tile = it.t_begin + i;
         const bool doc = tile < it.n_doc_tiles;
+        const int32_t page_id = next_page;
+        next_page = (tile + 1 < it.n_doc_tiles && lane < kPagesPerTile)
+                        ? load_page_id(p.batch, it.req, (tile + 1) * kPagesPerTile + lane)
+                        : -1;
         PageRef pg;
         pg.page = -1; pg.nvalid = 0; pg.lstart = 0;
         if (doc && lane < kPagesPerTile)
-          pg = page_ref(p.batch, it.req, tile * kPagesPerTile + lane, p.num_pages, p.err);
+          pg = page_ref_cached(&ctl->chunks, p.batch, it.req, tile * kPagesPerTile + lane, page_id, p.num_pages,
+                               p.err);
         const uint32_t slot = t % kIDescSlots;
         if (t >= kIDescSlots && !mbar_wait(&ctl->desc_empty[slot], ((t / kIDescSlots) - 1) & 1, abort_flag)) {
           bad = 1;
@@ -349,7 +392,7 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

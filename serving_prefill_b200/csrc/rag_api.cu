@@ -47,6 +47,16 @@ static cudaEvent_t take_event() {
   return e;
 }
 
+// Inside a stream capture the events become external event-record nodes of
+// the graph, which stay readable with cudaEventElapsedTime after each replay.
+static void record_event(cudaEvent_t ev, cudaStream_t stream) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, stream);
+}
+
 struct LaunchScope {
   int kind;
   cudaStream_t stream;
@@ -56,13 +66,13 @@ struct LaunchScope {
       std::lock_guard<std::mutex> lk(g_prof_mu);
       start = take_event();
       stop = take_event();
-      cudaEventRecord(start, stream);
+      record_event(start, stream);
     }
   }
   void done(cudaError_t e) {
     if (e == cudaSuccess) g_launches.fetch_add(1);
     if (start) {
-      cudaEventRecord(stop, stream);
+      record_event(stop, stream);
       std::lock_guard<std::mutex> lk(g_prof_mu);
       g_prof.push_back({kind, start, stop});
     }

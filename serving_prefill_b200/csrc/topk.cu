@@ -3,12 +3,14 @@
 // takes max(1, int(doc_token_count * ratio)) and torch.topk over the doc slice
 // of the impact vector).
 //
-// One CTA per request: an exact 4-pass radix select (8 bits per pass) over
-// the fp32 impact bits finds the k-th largest value T; the CTA then keeps
-// every doc token above T and the lowest-index tokens equal to T, and sorts
-// the k survivors by (impact descending, position ascending) with a bitonic
-// network in shared memory. Impacts are >= 0, so their IEEE bit patterns
-// order like the values.
+// One CTA per request. A histogram of the top 12 bits of the fp32 impacts
+// (impacts are >= 0, so their bit patterns order like the values) finds the
+// bucket holding the k-th largest value; keys above it are scattered into
+// their buckets' ranges in descending bucket order, and the keys inside it
+// become candidates. Candidates and each bucket's keys are then ordered by
+// counting ranks of the composite key (impact descending, position
+// ascending); a bitonic network in shared memory takes over for long runs,
+// and an exact radix select handles a bucket too full to stage.
 #include <cuda_runtime.h>
 
 #include "params.cuh"
@@ -20,6 +22,7 @@ constexpr int kTopkBins = 4096;
 constexpr int kBatch = 8;    // keys in flight per thread per radix pass
 constexpr int kTopkMaxSort = 8192;   // requests up to this many doc tokens are sorted whole
 constexpr int kTopkCand = 8192;      // candidates of the k-th key's bucket kept in shared memory
+constexpr int kTopkRankMax = 512;    // runs up to this long are ordered by counting ranks
 
 
 __device__ __forceinline__ uint32_t impact_key(float v) {
@@ -101,8 +104,10 @@ __device__ __forceinline__ void digit_histogram(const float* keys, int n, uint32
 
 // The digit holding the kr-th largest key (counting from the top bin down):
 // sel[0] = digit, sel[1] = rank of the wanted key inside that digit's bin.
+// When `start` is given it receives, per bin, the number of keys in the bins
+// above it (where that bin's keys begin in descending order).
 __device__ __forceinline__ void select_digit(const uint32_t* hist, int nbins, uint32_t kr, uint32_t* sel,
-                                             int* warp_sums) {
+                                             int* warp_sums, uint32_t* start) {
   const int tid = threadIdx.x;
   const int per = nbins / kTopkThreads > 0 ? nbins / kTopkThreads : 1;
   const int hi_bin = nbins - 1 - tid * per;     // this thread's bins: hi_bin .. hi_bin - per + 1
@@ -111,22 +116,32 @@ __device__ __forceinline__ void select_digit(const uint32_t* hist, int nbins, ui
     for (int j = 0; j < per; ++j) mine += hist[hi_bin - j];
   const int incl = block_scan_incl(int(mine), warp_sums);
   const uint32_t before = uint32_t(incl) - mine;
-  if (tid * per < nbins && before < kr && uint32_t(incl) >= kr) {
+  if (tid * per < nbins) {
     uint32_t cum = before;
+    bool found = !(before < kr && uint32_t(incl) >= kr);
     for (int j = 0; j < per; ++j) {
       const uint32_t h = hist[hi_bin - j];
-      if (cum + h >= kr) { sel[0] = uint32_t(hi_bin - j); sel[1] = kr - cum; break; }
+      if (start) start[hi_bin - j] = cum;
+      if (!found && cum + h >= kr) { sel[0] = uint32_t(hi_bin - j); sel[1] = kr - cum; found = true; }
       cum += h;
     }
   }
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkParams p) {
+// Position of composite key c among the sorted run a[s, e) of distinct keys.
+__device__ __forceinline__ int rank_in(const uint64_t* a, int s, int e, uint64_t c) {
+  int r = 0;
+  for (int j = s; j < e; ++j) r += a[j] < c;
+  return r;
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams p) {
   extern __shared__ uint64_t smem_topk[];
-  uint64_t* sort_buf = smem_topk;                  // [kTopkMaxSort]
-  uint64_t* cand = smem_topk + kTopkMaxSort;       // [kTopkCand]
+  uint64_t* sel_buf = smem_topk;                   // [kTopkMaxSort] selected keys, grouped by bucket
+  uint64_t* cand = smem_topk + kTopkMaxSort;       // [kTopkCand] keys of the k-th key's bucket
   __shared__ uint32_t hist[kTopkBins];
+  __shared__ uint32_t pos[kTopkBins];
   __shared__ uint32_t s_sel[2];
   __shared__ uint32_t s_cnt[2];
   __shared__ int warp_sums[32];
@@ -147,98 +162,125 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkParams p) 
   }
   if (k == 0) return;
 
-  int kp = 1;
-  if (n <= kTopkMaxSort) {
-    // ---- short request: sort every doc token
-    while (kp < n) kp <<= 1;
-    for (int i = tid; i < kp; i += kTopkThreads) sort_buf[i] = i < n ? composite(impact_key(keys[i]), i) : ~0ull;
-    __syncthreads();
-    bitonic_sort(sort_buf, kp);
-  } else {
-    // ---- long request. Pass 1: the 12-bit bucket (sign, exponent, 3 mantissa
-    // bits) that holds the k-th largest key, and how many keys lie above it.
-    digit_histogram(keys, n, 0u, 0u, 20, kTopkBins, hist);
-    select_digit(hist, kTopkBins, uint32_t(k), s_sel, warp_sums);
-    const uint32_t d1 = s_sel[0];
-    const int kr1 = int(s_sel[1]);
-    const int n_gt1 = k - kr1;
-    if (tid == 0) { s_cnt[0] = 0; s_cnt[1] = 0; }
-    __syncthreads();
-    // Pass 2: keys above the bucket go straight to the output buffer; keys in
-    // it are gathered as candidates.
-    for (int base = 0; base < n; base += kTopkThreads * kBatch) {
-      uint32_t u[kBatch];
+  // Pass 1: histogram of the 12-bit buckets (sign, exponent, 3 mantissa bits);
+  // d1 is the bucket of the k-th largest key, kr1 its rank inside it, and
+  // pos[d] where bucket d's keys start in descending order.
+  digit_histogram(keys, n, 0u, 0u, 20, kTopkBins, hist);
+  select_digit(hist, kTopkBins, uint32_t(k), s_sel, warp_sums, pos);
+  const uint32_t d1 = s_sel[0];
+  const int kr1 = int(s_sel[1]);
+  const int n_gt1 = k - kr1;
+  if (tid == 0) { s_cnt[0] = 0; s_cnt[1] = 0; }
+  __syncthreads();
+  // Pass 2: keys above bucket d1 go to their bucket's range of sel_buf; keys
+  // in d1 are gathered as candidates.
+  for (int base = 0; base < n; base += kTopkThreads * kBatch) {
+    uint32_t u[kBatch];
 #pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int i = base + j * kTopkThreads + tid;
-        u[j] = i < n ? impact_key(__ldg(keys + i)) : 0u;
-      }
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = base + j * kTopkThreads + tid;
+      u[j] = i < n ? impact_key(__ldg(keys + i)) : 0u;
+    }
 #pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int i = base + j * kTopkThreads + tid;
-        if (i >= n) continue;
-        const uint32_t dig = u[j] >> 20;
-        if (dig > d1) {
-          sort_buf[atomicAdd(&s_cnt[0], 1u)] = composite(u[j], i);
-        } else if (dig == d1) {
-          const uint32_t c = atomicAdd(&s_cnt[1], 1u);
-          if (c < uint32_t(kTopkCand)) cand[c] = composite(u[j], i);
-        }
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = base + j * kTopkThreads + tid;
+      if (i >= n) continue;
+      const uint32_t dig = u[j] >> 20;
+      if (dig > d1) {
+        sel_buf[atomicAdd(&pos[dig], 1u)] = composite(u[j], i);
+      } else if (dig == d1) {
+        const uint32_t c = atomicAdd(&s_cnt[1], 1u);
+        if (c < uint32_t(kTopkCand)) cand[c] = composite(u[j], i);
       }
     }
-    __syncthreads();
-    const int nc = int(s_cnt[1]);
-    if (nc <= kTopkCand) {
-      // Sort the candidates (ties by position) and keep the best kr1.
+  }
+  __syncthreads();
+  const int nc = int(s_cnt[1]);
+
+  if (nc <= kTopkCand) {
+    // the best kr1 candidates, in order, after the keys of the buckets above
+    if (nc <= kTopkRankMax) {
+      for (int i = tid; i < nc; i += kTopkThreads) {
+        const uint64_t c = cand[i];
+        const int r = rank_in(cand, 0, nc, c);
+        if (r < kr1) sel_buf[n_gt1 + r] = c;
+      }
+    } else {
       int cp = 1;
       while (cp < nc) cp <<= 1;
       for (int i = nc + tid; i < cp; i += kTopkThreads) cand[i] = ~0ull;
       __syncthreads();
       bitonic_sort(cand, cp);
-      for (int i = tid; i < kr1; i += kTopkThreads) sort_buf[n_gt1 + i] = cand[i];
-    } else {
-      // Too many keys share the bucket: exact radix select on the low 20 bits
-      // over global memory, then index-ordered compaction.
-      uint32_t prefix = d1 << 20, mask = 0xfff00000u, kr = uint32_t(kr1);
-      for (int pass = 0; pass < 2; ++pass) {
-        const int shift = pass == 0 ? 8 : 0;
-        const int bits = pass == 0 ? 12 : 8;
-        const int nbins = 1 << bits;
-        digit_histogram(keys, n, prefix, mask, shift, nbins, hist);
-        select_digit(hist, nbins, kr, s_sel, warp_sums);
-        prefix |= s_sel[0] << shift;
-        mask |= uint32_t(nbins - 1) << shift;
-        kr = s_sel[1];
-        __syncthreads();
-      }
-      const uint32_t T = prefix;
-      const int n_gt = k - int(kr);
-      if (tid == 0) { s_sel[0] = uint32_t(n_gt1); s_sel[1] = 0; }   // keys > T already placed: those above d1
-      __syncthreads();
-      for (int base = 0; base < n; base += kTopkThreads) {
-        const int i = base + tid;
-        const uint32_t u = i < n ? impact_key(__ldg(keys + i)) : 0u;
-        const bool in_bucket = i < n && (u >> 20) == d1;
-        const bool gt = in_bucket && u > T;
-        const bool eq = in_bucket && u == T;
-        if (gt) sort_buf[atomicAdd(&s_sel[0], 1u)] = composite(u, i);
-        const int eq_incl = block_scan_incl(eq ? 1 : 0, warp_sums);
-        const uint32_t seen = s_sel[1];
-        const uint32_t rank = seen + uint32_t(eq_incl) - (eq ? 1u : 0u);
-        if (eq && rank < kr) sort_buf[n_gt + rank] = composite(u, i);
-        __syncthreads();
-        if (tid == kTopkThreads - 1) s_sel[1] = seen + uint32_t(eq_incl);
-        __syncthreads();
-        if (s_sel[1] >= kr && s_sel[0] >= uint32_t(n_gt)) break;
-      }
+      for (int i = tid; i < kr1; i += kTopkThreads) sel_buf[n_gt1 + i] = cand[i];
     }
-    while (kp < k) kp <<= 1;
-    for (int i = k + tid; i < kp; i += kTopkThreads) sort_buf[i] = ~0ull;
     __syncthreads();
-    bitonic_sort(sort_buf, kp);
+    // keys above d1: each lands at its bucket's start plus its rank in the bucket
+    bool small_buckets = true;
+    for (int d = tid; d < kTopkBins; d += kTopkThreads)
+      if (d > int(d1) && hist[d] > uint32_t(kTopkRankMax)) small_buckets = false;
+    if (__syncthreads_and(small_buckets ? 1 : 0)) {
+      for (int i = tid; i < k; i += kTopkThreads) {
+        const uint64_t c = sel_buf[i];
+        int at = i;
+        if (i < n_gt1) {
+          const uint32_t d = (~uint32_t(c >> 32)) >> 20;
+          const int e = int(pos[d]);
+          const int s0 = e - int(hist[d]);
+          at = s0 + rank_in(sel_buf, s0, e, c);
+        }
+        out_idx[at] = int32_t(c & 0xffffffffu);
+        if (out_val) out_val[at] = __uint_as_float(~uint32_t(c >> 32));
+      }
+      return;
+    }
+    int kp = 1;
+    while (kp < k) kp <<= 1;
+    for (int i = k + tid; i < kp; i += kTopkThreads) sel_buf[i] = ~0ull;
+    __syncthreads();
+    bitonic_sort(sel_buf, kp);
+  } else {
+    // Too many keys share bucket d1: exact radix select on its low 20 bits over
+    // global memory, then index-ordered compaction and a full sort.
+    uint32_t prefix = d1 << 20, mask = 0xfff00000u, kr = uint32_t(kr1);
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = pass == 0 ? 8 : 0;
+      const int bits = pass == 0 ? 12 : 8;
+      const int nbins = 1 << bits;
+      digit_histogram(keys, n, prefix, mask, shift, nbins, hist);
+      select_digit(hist, nbins, kr, s_sel, warp_sums, nullptr);
+      prefix |= s_sel[0] << shift;
+      mask |= uint32_t(nbins - 1) << shift;
+      kr = s_sel[1];
+      __syncthreads();
+    }
+    const uint32_t T = prefix;
+    const int n_gt = k - int(kr);
+    if (tid == 0) { s_sel[0] = uint32_t(n_gt1); s_sel[1] = 0; }   // keys above d1 are already placed
+    __syncthreads();
+    for (int base = 0; base < n; base += kTopkThreads) {
+      const int i = base + tid;
+      const uint32_t u = i < n ? impact_key(__ldg(keys + i)) : 0u;
+      const bool in_bucket = i < n && (u >> 20) == d1;
+      const bool gt = in_bucket && u > T;
+      const bool eq = in_bucket && u == T;
+      if (gt) sel_buf[atomicAdd(&s_sel[0], 1u)] = composite(u, i);
+      const int eq_incl = block_scan_incl(eq ? 1 : 0, warp_sums);
+      const uint32_t seen = s_sel[1];
+      const uint32_t rank = seen + uint32_t(eq_incl) - (eq ? 1u : 0u);
+      if (eq && rank < kr) sel_buf[n_gt + rank] = composite(u, i);
+      __syncthreads();
+      if (tid == kTopkThreads - 1) s_sel[1] = seen + uint32_t(eq_incl);
+      __syncthreads();
+      if (s_sel[1] >= kr && s_sel[0] >= uint32_t(n_gt)) break;
+    }
+    int kp = 1;
+    while (kp < k) kp <<= 1;
+    for (int i = k + tid; i < kp; i += kTopkThreads) sel_buf[i] = ~0ull;
+    __syncthreads();
+    bitonic_sort(sel_buf, kp);
   }
   for (int i = tid; i < k; i += kTopkThreads) {
-    const uint64_t comp = sort_buf[i];
+    const uint64_t comp = sel_buf[i];
     out_idx[i] = int32_t(comp & 0xffffffffu);
     if (out_val) out_val[i] = __uint_as_float(~uint32_t(comp >> 32));
   }
@@ -246,7 +288,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkParams p) 
 
 cudaError_t launch_topk(const TopkParams& p, int num_requests, int max_k, cudaStream_t stream) {
   (void)max_k;
-  const size_t smem = sizeof(uint64_t) * size_t(kTopkMaxSort + kTopkCand);
+  const size_t smem = sizeof(uint64_t) * size_t(kTopkMaxSort + kTopkCand);   // + 32 KB static
   static size_t attr_set = 0;   // largest dynamic smem size configured so far
   if (smem > attr_set) {
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
