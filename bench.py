@@ -404,17 +404,28 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_step(w, lay, layer_inputs, heads):
-    """The oracle on a sample of query heads of every layer, then top-k."""
+def oracle_step(w, lay, layer_inputs, groups):
+    """The oracle on a sample of KV-head groups of every layer, then top-k.
+
+    A group is one KV head with the G query heads that read it, so a sample
+    of n groups is the same problem with n KV heads: its pool, gather and
+    attention all shrink in proportion.
+    """
     import oracle.prefill as orc
     scale = 1.0 / np.sqrt(w.head_dim)
     bits = np.uint16 if w.dtype == "bf16" else np.uint32
+    G = w.num_q_heads // w.num_kv_heads
+    heads = [g * G + j for g in groups for j in range(G)]
     impact_all = None
     for layer in range(w.num_layers):
         inp = layer_inputs[layer]
-        pk, pv = orc.build_layer_pool(lay, inp, bits)
-        q_all, kq_all, vq_all = orc.to_f64(inp.q), orc.to_f64(inp.kq), orc.to_f64(inp.vq)
-        G = w.num_q_heads // w.num_kv_heads
+        pk = orc.new_pool(1, lay.num_pages, len(groups), w.head_dim, bits)
+        pv = orc.new_pool(1, lay.num_pages, len(groups), w.head_dim, bits)
+        for c, pages in enumerate(lay.chunk_pages):
+            orc.pool_write(pk, 0, pages.numpy(), orc.to_bits(inp.chunk_k[c][:, groups]))
+            orc.pool_write(pv, 0, pages.numpy(), orc.to_bits(inp.chunk_v[c][:, groups]))
+        q_all = orc.to_f64(inp.q[:, heads])
+        kq_all, vq_all = orc.to_f64(inp.kq[:, groups]), orc.to_f64(inp.vq[:, groups])
         q0 = 0
         imps = []
         for b, cs in enumerate(lay.req_chunks):
@@ -425,12 +436,7 @@ def oracle_step(w, lay, layer_inputs, heads):
             n_doc = kd.shape[0]
             kcat = np.concatenate([kd, kq_all[q0:q0 + ql]])
             vcat = np.concatenate([vd, vq_all[q0:q0 + ql]])
-            sel_q = q_all[q0:q0 + ql][:, heads, :]
-            kv_heads = sorted({h // G for h in heads})
-            remap = [kv_heads.index(h // G) for h in heads]
-            ks = kcat[:, kv_heads, :][:, remap, :]
-            vs = vcat[:, kv_heads, :][:, remap, :]
-            _, _, _, imp, _ = orc.attend_request(sel_q, ks, vs, n_doc, scale,
+            _, _, _, imp, _ = orc.attend_request(q_all[q0:q0 + ql], kcat, vcat, n_doc, scale,
                                                  want_impact=(layer == w.impact_layer_index))
             if imp is not None:
                 k = orc.recompute_count(n_doc, w.r)
@@ -446,23 +452,25 @@ def run_reference(args, w, budget_per_step=None):
     lay = make_layout(w)
     layer_inputs = [make_layer_inputs(w, lay, layer) for layer in range(w.num_layers)]
     doc = sum(lay.doc_lens)
-    # calibrate: one head of every layer
+    # calibrate on one KV-head group of every layer
     t0 = time.perf_counter()
     oracle_step(w, lay, layer_inputs, [0])
-    t_head = max(time.perf_counter() - t0, 1e-3)
+    t_group = max(time.perf_counter() - t0, 1e-3)
     budget = budget_per_step or max(0.5, 150.0 / max(1, args.steps + args.warmup))
-    n_heads = int(max(1, min(w.num_q_heads, budget // t_head)))
-    heads = list(range(0, w.num_q_heads, max(1, w.num_q_heads // n_heads)))[:n_heads]
+    n = int(max(1, min(w.num_kv_heads, budget // t_group)))
+    groups = list(range(0, w.num_kv_heads, max(1, w.num_kv_heads // n)))[:n]
     for _ in range(args.warmup):
-        oracle_step(w, lay, layer_inputs, heads)
+        oracle_step(w, lay, layer_inputs, groups)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(w, lay, layer_inputs, heads)
+        oracle_step(w, lay, layer_inputs, groups)
     dt = time.perf_counter() - t0
-    frac = len(heads) / w.num_q_heads
+    frac = len(groups) / w.num_kv_heads
     value = doc * frac * args.steps / dt
-    sample = (f"{len(heads)} of {w.num_q_heads} query heads of every layer (gather, attention, impact, "
-              f"top-k over all doc tokens); tokens/s scaled by the head fraction")
+    G = w.num_q_heads // w.num_kv_heads
+    sample = (f"{len(groups)} of {w.num_kv_heads} KV-head groups ({len(groups) * G} of {w.num_q_heads} query "
+              f"heads) of every layer: pool write, gather, attention, impact, top-k over all doc tokens; "
+              f"tokens/s scaled by the group fraction")
     return value, dt / args.steps, sample
 
 

@@ -30,7 +30,7 @@ constexpr int kIHalf = kITileBytes / 2;
 constexpr int kIQHalf = kImpactRows * 128;          // 256 rows x 64 d (bf16) per d-half
 constexpr int kIQBytes = 2 * kIQHalf;
 constexpr int kImpThreads = 320;              // 8 epilogue + producer + MMA warps
-constexpr int kImpPolyPairsOf8 = 3;          // of every 8 column pairs, 3 use the FMA-pipe exp2
+constexpr int kImpPolyPairsOf8 = 0;          // of every 8 column pairs, this many use the FMA-pipe exp2 (fastest: 0)
 
 struct ImpDesc {
   int32_t kind;      // 0 doc tile, 1 query-key tile
@@ -48,8 +48,7 @@ struct ImpCtrl {
   uint64_t desc_full[kIDescSlots], desc_empty[kIDescSlots];
   ImpDesc desc[kIDescSlots];
   ChunkCache chunks;
-  alignas(16) float neg_m2[kImpactRows];   // -m of every row of the block (log2 units; -inf: no row)
-  alignas(16) float il[kImpactRows];       // 1 / (l * H_q) of every row
+  alignas(16) float neg_m2[kImpactRows];   // per row: log2(1 / (l * H_q)) - m (log2 units; -inf: no row)
   float red[2][kBN];                      // second-half column sums, per S buffer
   uint32_t tmem_base;
   int32_t abort;
@@ -172,7 +171,6 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int half = warp >> 2;
     const int k = (warp & 3) * 32 + lane;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
-    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     uint32_t t_glob = 0;
     int bad = 0;
     for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
@@ -182,15 +180,16 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       named_bar_sync(1, 256);
       {
         const int r = tid;   // 256 epilogue threads, one row each
-        float nm = -INFINITY, iv = 0.f;
+        // per row: -m + log2(1 / (l * H_q)), so that 2^(s*c + bias) is the
+        // row's normalised weight already divided by H_q (-inf: no row)
+        float bias = -INFINITY;
         if (r < it.nrows) {
           const int pr = it.rb * kImpactRows + r;
           const int64_t row = int64_t(it.req.q0 + pr / G) * p.num_q_heads + it.g * G + pr % G;
-          nm = -p.row_m2[row];
-          iv = p.row_il[row];
+          const float il = p.row_il[row];
+          bias = il > 0.f ? __log2f(il) - p.row_m2[row] : -INFINITY;
         }
-        ctl->neg_m2[r] = nm;
-        ctl->il[r] = iv;
+        ctl->neg_m2[r] = bias;
       }
       named_bar_sync(1, 256);
       float* seg = p.impact + (it.req.doc0 + it.req.q0);
@@ -219,45 +218,45 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (lane == 0) mbar_arrive(&ctl->desc_empty[slot]);
         if (!mbar_wait(&ctl->s_full[buf], (t >> 1) & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
-        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         const uint32_t col = tmem + lane_off + (buf ? 256u : 0u) + c0;
-        for (int c = 0; c < cols; c += 32) {
-          uint32_t u[32];
-          tmem_ld32(col + c, u);
-          tmem_wait_ld();
+        // 32-column chunks with the next chunk's TMEM load in flight while
+        // the current one is reduced
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        auto chunk = [&](const uint32_t (&u)[32], int cbase) {
 #pragma unroll
           for (int j = 0; j < 32; j += 4) {
-            const int r0 = c0 + c + j;
-            const float4 nm = *reinterpret_cast<const float4*>(&ctl->neg_m2[r0]);
-            const float4 iv = *reinterpret_cast<const float4*>(&ctl->il[r0]);
-            const float2 x01 = ffma2(make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1])), sc2,
-                                     make_float2(nm.x, nm.y));
-            const float2 x23 = ffma2(make_float2(__uint_as_float(u[j + 2]), __uint_as_float(u[j + 3])), sc2,
-                                     make_float2(nm.z, nm.w));
-            float2 e01, e23;
-            if (((j >> 1) & 7) < kImpPolyPairsOf8) {
-              e01 = exp2_poly2(x01);
-            } else {
-              e01 = make_float2(ex2(x01.x), ex2(x01.y));
+            const int r0 = c0 + cbase + j;
+            const float4 bias = *reinterpret_cast<const float4*>(&ctl->neg_m2[r0]);
+            float e[4];
+            e[0] = fmaf(__uint_as_float(u[j]), p.scale_log2, bias.x);
+            e[1] = fmaf(__uint_as_float(u[j + 1]), p.scale_log2, bias.y);
+            e[2] = fmaf(__uint_as_float(u[j + 2]), p.scale_log2, bias.z);
+            e[3] = fmaf(__uint_as_float(u[j + 3]), p.scale_log2, bias.w);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float v = ((((j + q) >> 1) & 7) < kImpPolyPairsOf8) ? exp2_poly(e[q]) : ex2(e[q]);
+              if (kind != 0 && r0 + q < rlim) v = 0.f;
+              acc[q] += v;
             }
-            if ((((j >> 1) + 1) & 7) < kImpPolyPairsOf8) {
-              e23 = exp2_poly2(x23);
-            } else {
-              e23 = make_float2(ex2(x23.x), ex2(x23.y));
-            }
-            if (kind != 0) {
-              if (r0 < rlim) e01.x = 0.f;
-              if (r0 + 1 < rlim) e01.y = 0.f;
-              if (r0 + 2 < rlim) e23.x = 0.f;
-              if (r0 + 3 < rlim) e23.y = 0.f;
-            }
-            acc0 = ffma2(e01, make_float2(iv.x, iv.y), acc0);
-            acc1 = ffma2(e23, make_float2(iv.z, iv.w), acc1);
           }
+        };
+        uint32_t ua[32], ub[32];
+        tmem_ld32(col, ua);
+        tmem_wait_ld();
+        for (int c = 0; c < cols; c += 64) {
+          const bool more_b = c + 32 < cols;
+          if (more_b) tmem_ld32(col + c + 32, ub);
+          chunk(ua, c);
+          tmem_wait_ld();
+          if (!more_b) break;
+          const bool more_a = c + 64 < cols;
+          if (more_a) tmem_ld32(col + c + 64, ua);
+          chunk(ub, c + 32);
+          tmem_wait_ld();
         }
         tc_fence_before();
         mbar_arrive(&ctl->s_free[buf]);
-        float total = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+        float total = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         if (half == 1) ctl->red[buf][k] = total;
         named_bar_sync(2, 256);
         if (half == 0) {

@@ -12,7 +12,7 @@
 #include <mutex>
 #include <vector>
 
-#include "../../include/rag_prefill.h"
+#include "rag_prefill.h"
 #include "params.cuh"
 
 namespace rag {

@@ -12,7 +12,7 @@
 
 #include <mutex>
 
-#include "../../include/rag_prefill.h"
+#include "rag_prefill.h"
 
 namespace {
 
