@@ -25,6 +25,7 @@
 // hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "params.cuh"
@@ -147,6 +148,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int lane = tid & 31;
   const int B = p.batch.num_requests;
   const int G = p.group;
+
+  // the kernels after this one (combine, impact) may start launching now;
+  // they wait for this grid before they read what it writes
+  pdl_launch_dependents();
 
   // zero the impact accumulator for the impact pass that follows
   if (p.impact_zero) {
@@ -399,10 +404,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (p.row_lse) p.row_lse[row] = (m_use + __log2f(l_sum)) * 0.69314718055994531f;
         }
       } else {
-        float4* dst = reinterpret_cast<float4*>(p.part + ((size_t(w) * kQTiles + qt) * kBM + r) * kPartStride);
+        // partial row: this split's own softmax average O/l in fp16 (|O/l| is
+        // bounded by max |V|), then its reference max m and sum l in fp32
+        const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+        uint4* dst = reinterpret_cast<uint4*>(p.part + ((size_t(w) * kQTiles + qt) * kBM + r) * kPartStride);
 #pragma unroll
-        for (int c = 0; c < kHeadDim / 4; ++c) dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-        dst[kHeadDim / 4] = make_float4(m_ref, l_sum, 0.f, 0.f);
+        for (int c = 0; c < kHeadDim / 8; ++c) {
+          uint4 v;
+          v.x = pack_f16x2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
+          v.y = pack_f16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
+          v.z = pack_f16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
+          v.w = pack_f16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
+          dst[c] = v;
+        }
+        reinterpret_cast<float4*>(dst + kHeadDim / 8)[0] = make_float4(m_ref, l_sum, 0.f, 0.f);
       }
     }
     if (bad) raise_abort(ctl, p.err);
@@ -644,6 +659,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 constexpr int kCombineRowsPerBlock = 8;
 
 __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p, int max_rb) {
+  pdl_launch_dependents();
+  pdl_wait();   // partials and item offsets come from the forward kernel
   const int groups = kFwdRows / kCombineRowsPerBlock;
   const int b = blockIdx.y;
   const int unit = blockIdx.x / groups;
@@ -663,13 +680,15 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p
   const size_t first = size_t(base) + size_t(g) * sh.n_split * sh.n_rt + rb;
   if (first + size_t(sh.n_split - 1) * sh.n_rt >= size_t(p.max_items)) return;
   // statistics of every split first (lane s holds split s, 32 at a time), then
-  // the weighted rows with several loads in flight
+  // the weighted rows with several loads in flight; split s weighs its own
+  // average O_s/l_s by l_s * 2^(m_s - m)
   const float* row0 = p.part + (first * kFwdRows + rr) * kPartStride;
   const size_t split_stride = size_t(sh.n_rt) * kFwdRows * kPartStride;
+  constexpr int kStatOff = kHeadDim / 2;   // 32-bit word of m (then l) in a row
   float m = -INFINITY;
   for (int s0 = 0; s0 < sh.n_split; s0 += 32) {
     const int s = s0 + lane;
-    const float ms = s < sh.n_split ? __ldcg(row0 + s * split_stride + kHeadDim) : -INFINITY;
+    const float ms = s < sh.n_split ? __ldcg(row0 + s * split_stride + kStatOff) : -INFINITY;
     float mm = ms;
     for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
     m = fmaxf(m, mm);
@@ -678,24 +697,26 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p
   float l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s0 = 0; s0 < sh.n_split; s0 += 8) {
-    float4 v[8];
+    uint2 v[8];
     float2 ml[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (s0 + j < sh.n_split) {
         const float* row = row0 + (s0 + j) * split_stride;
-        ml[j] = __ldcg(reinterpret_cast<const float2*>(row + kHeadDim));
-        v[j] = __ldcg(reinterpret_cast<const float4*>(row) + lane);
+        ml[j] = __ldcg(reinterpret_cast<const float2*>(row + kStatOff));
+        v[j] = __ldcg(reinterpret_cast<const uint2*>(row) + lane);
       } else {
         ml[j] = make_float2(-INFINITY, 0.f);
-        v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        v[j] = make_uint2(0u, 0u);
       }
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float wgt = (ml[j].x == -INFINITY) ? 0.f : ex2(ml[j].x - m_use);
-      l += ml[j].y * wgt;
-      acc.x += v[j].x * wgt; acc.y += v[j].y * wgt; acc.z += v[j].z * wgt; acc.w += v[j].w * wgt;
+      const float wgt = (ml[j].x == -INFINITY) ? 0.f : ml[j].y * ex2(ml[j].x - m_use);
+      const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&v[j].x));
+      const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&v[j].y));
+      l += wgt;
+      acc.x += lo.x * wgt; acc.y += lo.y * wgt; acc.z += hi.x * wgt; acc.w += hi.y * wgt;
     }
   }
   const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -729,8 +750,7 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
 
 cudaError_t launch_attn_combine(const CombineParams& p, int max_rb, int num_requests, cudaStream_t stream) {
   dim3 grid(p.num_kv_heads * max_rb * (kFwdRows / kCombineRowsPerBlock), num_requests);
-  attn_combine_kernel<<<grid, 256, 0, stream>>>(p, max_rb);
-  return cudaGetLastError();
+  return launch_pdl(attn_combine_kernel, grid, dim3(256), 0, stream, 1, p, max_rb);
 }
 
 }  // namespace rag

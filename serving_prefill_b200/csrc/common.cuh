@@ -18,7 +18,7 @@ constexpr int kBN = 128;              // keys per tile
 constexpr int kPagesPerTile = kBN / kPage;
 constexpr int kImpactRows = 256;      // rows per impact-pass block (MMA N)
 constexpr int kMaxRequests = 4096;
-constexpr int kPartStride = 132;      // floats per partial row: O[128], m, l, pad
+constexpr int kPartStride = 68;       // 32-bit words per partial row: O/l as 64 fp16 pairs, m, l, pad
 
 // device error word bits (rag_last_device_error reports them)
 enum : int32_t {
@@ -215,7 +215,7 @@ __device__ __forceinline__ PageRef page_ref_cached(const ChunkCache* cc, const B
 //   item prefix                (kMaxRequests + 1) int32
 //   row_m2                     total_q * H_q fp32   (reference max, log2 units)
 //   row_il                     total_q * H_q fp32   (1 / (l * H_q))
-//   partials                   items * 256 * kPartStride fp32
+//   partials                   items * 256 * kPartStride 32-bit words
 struct WsLayout {
   size_t off_prefix, off_m2, off_il, off_part, total;
 };

@@ -119,6 +119,7 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = p.batch.num_requests;
   const int G = p.group;
+  pdl_launch_dependents();
 
   if (tid == 0) {
     mbar_init(&ctl->q_full, 1);
@@ -173,6 +174,10 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     uint32_t t_glob = 0;
     int bad = 0;
+    // The row statistics, and the zeroed impact vector, come from the kernels
+    // before this one; the producer and MMA warps only read inputs and start
+    // on the first tiles while those finish.
+    pdl_wait();
     for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
       const ImpItem it = decode_imp_item(p, prefix, w);
       const int n = it.t_end - it.t_begin;
@@ -406,8 +411,7 @@ cudaError_t launch_impact(const CUtensorMap& tq, const CUtensorMap& tk, const CU
     if (e != cudaSuccess) return e;
     attr_set = smem;
   }
-  impact_kernel<<<grid, kImpThreads, smem, stream>>>(tq, tk, tkq, p);
-  return cudaGetLastError();
+  return launch_pdl(impact_kernel, dim3(grid), dim3(kImpThreads), smem, stream, 1, tq, tk, tkq, p);
 }
 
 }  // namespace rag

@@ -139,15 +139,21 @@ static Plan plan_split(const rag_batch& b, int num_kv_heads, int group, int rows
   const int tiles_avg = std::max(1, cdiv(int64_t(std::ceil(avg_pages)), kPagesPerTile) +
                                         cdiv(int64_t(std::ceil(avg_q)), kBN));
   const double units = double(num_kv_heads) * B * rt_avg;
+  // Every split length from 2 tiles to the whole row, with a fixed cost per
+  // item (Q load, pipeline fill and the partial-row epilogue, about three
+  // tiles' worth). One request: its items are alike, and the busiest SM runs
+  // ceil(items / sms) of them. Several requests: items differ in length and
+  // are dealt out round-robin, so the estimate is the list-scheduling bound,
+  // the average load per SM plus one longest item.
+  constexpr double kItemOverheadTiles = 3.0;
+  const double total_tiles = units * tiles_avg;
   double best = 1e300;
-  int best_ts = tiles_max;
-  for (int waves = 1; waves <= 32; ++waves) {
-    const double target = double(sms) * waves;
-    int ts = std::max(2, int(std::ceil(units * tiles_avg / target)));
-    ts = std::min(ts, std::max(tiles_max, 1));
+  int best_ts = std::max(tiles_max, 1);
+  for (int ts = std::min(2, std::max(tiles_max, 1)); ts <= std::max(tiles_max, 1); ++ts) {
     const double items = units * std::ceil(double(tiles_avg) / ts);
-    const double cost = std::ceil(items / sms) * (ts + 2.0);
-    if (cost < best - 1e-9 || (std::fabs(cost - best) < 1e-9 && ts > best_ts)) {
+    const double cost = B == 1 ? std::ceil(items / sms) * (ts + kItemOverheadTiles)
+                               : (total_tiles + items * kItemOverheadTiles) / sms + ts + kItemOverheadTiles;
+    if (cost < best + 1e-9) {   // ties go to the longer split (fewer partial rows)
       best = cost;
       best_ts = ts;
     }
