@@ -452,13 +452,24 @@ def run_reference(args, w, budget_per_step=None):
     lay = make_layout(w)
     layer_inputs = [make_layer_inputs(w, lay, layer) for layer in range(w.num_layers)]
     doc = sum(lay.doc_lens)
-    # calibrate on one KV-head group of every layer
-    t0 = time.perf_counter()
-    oracle_step(w, lay, layer_inputs, [0])
-    t_group = max(time.perf_counter() - t0, 1e-3)
+    # Calibrate: double the number of KV-head groups (spread over the heads)
+    # while one step still fits the per-step budget; the oracle's cost per
+    # group depends on how many groups it holds, so it is measured, not
+    # extrapolated. When the whole workload fits, every group is timed.
     budget = budget_per_step or max(0.5, 150.0 / max(1, args.steps + args.warmup))
-    n = int(max(1, min(w.num_kv_heads, budget // t_group)))
-    groups = list(range(0, w.num_kv_heads, max(1, w.num_kv_heads // n)))[:n]
+
+    def spread(n):
+        return list(range(0, w.num_kv_heads, max(1, w.num_kv_heads // n)))[:n]
+
+    n = 1
+    while n < w.num_kv_heads:
+        n2 = min(2 * n, w.num_kv_heads)
+        t0 = time.perf_counter()
+        oracle_step(w, lay, layer_inputs, spread(n2))
+        if time.perf_counter() - t0 > budget:
+            break
+        n = n2
+    groups = spread(n)
     for _ in range(args.warmup):
         oracle_step(w, lay, layer_inputs, groups)
     t0 = time.perf_counter()
