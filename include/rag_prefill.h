@@ -34,6 +34,10 @@
  *     never trapped, and reported by rag_last_device_error.
  *   - Indices of doc tokens are logical positions within their request,
  *     0 .. N_doc,b - 1, in concatenation order.
+ *   - Stream order holds as usual. The kernels are launched with programmatic
+ *     stream serialization: a kernel may begin its set-up (shared memory,
+ *     tensor memory) while the previous kernel in the stream finishes, but it
+ *     reads and writes global memory only after that kernel has completed.
  */
 #ifndef RAG_PREFILL_H_
 #define RAG_PREFILL_H_

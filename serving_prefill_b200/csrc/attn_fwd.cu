@@ -153,13 +153,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // they wait for this grid before they read what it writes
   pdl_launch_dependents();
 
-  // zero the impact accumulator for the impact pass that follows
-  if (p.impact_zero) {
-    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + tid; i < p.impact_len;
-         i += int64_t(gridDim.x) * blockDim.x)
-      p.impact_zero[i] = 0.f;
-  }
-
   if (tid == 0) {
     mbar_init(&ctl->q_full, 1);
     mbar_init(&ctl->q_empty, 1);
@@ -191,6 +184,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_kq);
   }
   if (warp == 9 && lane == 0) { tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_vq); }
+
+  // Everything above touches only this CTA's shared memory, TMEM and the
+  // kernel parameters, so it may overlap the previous kernel in the stream;
+  // from here on global memory is read and written, after that kernel ends.
+  pdl_wait();
+
+  // zero the impact accumulator for the impact pass that follows
+  if (p.impact_zero) {
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + tid; i < p.impact_len;
+         i += int64_t(gridDim.x) * blockDim.x)
+      p.impact_zero[i] = 0.f;
+  }
 
   // per-request item counts -> exclusive prefix (warp 0), total in ctl
   if (warp == 0) {
@@ -660,7 +665,8 @@ constexpr int kCombineRowsPerBlock = 8;
 
 __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p, int max_rb) {
   pdl_launch_dependents();
-  pdl_wait();   // partials and item offsets come from the forward kernel
+  // everything up to the item offset depends on the batch descriptors only,
+  // so it runs while the forward kernel finishes
   const int groups = kFwdRows / kCombineRowsPerBlock;
   const int b = blockIdx.y;
   const int unit = blockIdx.x / groups;
@@ -676,7 +682,8 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p
   const int tok = pr / G;
   if (tok >= req.n_q) return;
   const int head = g * G + pr % G;
-  const int base = p.item_prefix[b];
+  pdl_wait();   // partials and item offsets come from the forward kernel
+  const int base = __ldcg(p.item_prefix + b);
   const size_t first = size_t(base) + size_t(g) * sh.n_split * sh.n_rt + rb;
   if (first + size_t(sh.n_split - 1) * sh.n_rt >= size_t(p.max_items)) return;
   // statistics of every split first (lane s holds split s, 32 at a time), then
@@ -744,8 +751,7 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
     if (e != cudaSuccess) return e;
     attr_set = smem;
   }
-  attn_fwd_kernel<<<grid, kFwdThreads, smem, stream>>>(tq, tk, tv, tkq, tvq, p);
-  return cudaGetLastError();
+  return launch_pdl(attn_fwd_kernel, dim3(grid), dim3(kFwdThreads), smem, stream, 1, tq, tk, tv, tkq, tvq, p);
 }
 
 cudaError_t launch_attn_combine(const CombineParams& p, int max_rb, int num_requests, cudaStream_t stream) {
