@@ -65,3 +65,31 @@ def test_k_one_and_large_ratio():
     rng = np.random.default_rng(4)
     check([rng.random(15), rng.random(9)], 0.1)          # k = 1
     check([rng.random(12000)], 0.6)                       # k = 7200
+
+
+def test_cluster_of_four_ctas():
+    rng = np.random.default_rng(5)
+    check([rng.lognormal(-5, 1.5, 30000), rng.random(100)], 0.1)   # longest 30,000: four CTAs per request
+
+
+def test_buckets_at_the_rank_limit():
+    # one 12-bit bucket of 256 keys (ordered by counting) above one of 257 keys
+    # (ordered by a sorting network), both inside the top k
+    rng = np.random.default_rng(6)
+    y = 1.25 + 0.125 * rng.random(256)        # [1.25, 1.375): one bucket
+    x = 1.0 + 0.125 * rng.random(257)         # [1.0, 1.125): the bucket below it
+    low = 0.5 * rng.random(5000)
+    seg = np.concatenate([low[:2000], y, low[2000:], x])
+    n = len(seg)
+    check([seg], 600.5 / n)                    # k = 600: both buckets and 87 lower keys
+
+
+def test_large_buckets_use_wide_sorts():
+    rng = np.random.default_rng(7)
+    check([rng.random(65536)], 0.1)            # buckets of ~4,096 keys
+    check([rng.random(131072)], 0.05)          # the top bucket holds ~8,192 keys
+
+
+def test_many_buckets_across_the_cluster():
+    rng = np.random.default_rng(8)
+    check([rng.lognormal(-6, 2.5, 65536)], 0.1)   # hundreds of buckets dealt over eight CTAs
