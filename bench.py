@@ -67,7 +67,7 @@ def step_work(w, lay):
         "impact_flops_per_launch": impact_flops,
         "impact_bytes_per_launch": impact_bytes,
         "step_flops": attn_flops * L,
-        "step_bytes": per_layer_attn_bytes * L + imp_bytes * 2,
+        "step_bytes": per_layer_attn_bytes * L + (imp_bytes * 2 if w.select else 0),
         "doc_tokens": sum(lay.doc_lens),
     }
 
@@ -354,7 +354,7 @@ def run_e2e(args, w, lay, layer_inputs, rep, device, world):
     host_o = [torch.empty_like(o, device="cpu").pin_memory() for o in rep.outs]
     h2d = sum(t.numel() * t.element_size() for trip in host_in for t in trip) + sum(
         t.numel() * t.element_size() for t in desc)
-    d2h = host_topk.numel() * 4 + sum(o.numel() * o.element_size() for o in host_o)
+    d2h = (host_topk.numel() * 4 if w.select else 0) + sum(o.numel() * o.element_size() for o in host_o)
     steps = max(3, min(args.steps, 50))
 
     def one():
@@ -371,8 +371,9 @@ def run_e2e(args, w, lay, layer_inputs, rep, device, world):
                                    impact=eng.impact if layer == w.impact_layer_index else None,
                                    row_lse=eng.row_lse)
             host_o[layer].copy_(rep.outs[layer], non_blocking=True)
-        rag_impact_topk(eng.impact, rep.batch, w.r, eng.k_cap, eng.topk_idx, eng.topk_val, eng.k)
-        host_topk.copy_(eng.topk_idx, non_blocking=True)
+        if w.select:
+            rag_impact_topk(eng.impact, rep.batch, w.r, eng.k_cap, eng.topk_idx, eng.topk_val, eng.k)
+            host_topk.copy_(eng.topk_idx, non_blocking=True)
 
     for _ in range(3):
         one()
@@ -479,8 +480,9 @@ def run_reference(args, w, budget_per_step=None):
     frac = len(groups) / w.num_kv_heads
     value = doc * frac * args.steps / dt
     G = w.num_q_heads // w.num_kv_heads
+    what = "attention, impact, top-k over all doc tokens" if w.select else "attention (decode step)"
     sample = (f"{len(groups)} of {w.num_kv_heads} KV-head groups ({len(groups) * G} of {w.num_q_heads} query "
-              f"heads) of every layer: pool write, gather, attention, impact, top-k over all doc tokens; "
+              f"heads) of every layer: pool write, gather, {what}; "
               f"tokens/s scaled by the group fraction")
     return value, dt / args.steps, sample
 
@@ -557,7 +559,7 @@ def main():
             "config": {"workload": w.name, "requests": lay.num_requests, "layers": w.num_layers,
                        "doc_tokens_per_step": sum(lay.doc_lens), "query_tokens_per_step": lay.total_q,
                        "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
-                       "r": w.r, "parallelism": f"replicas x{world}",
+                       "r": w.r if w.select else None, "parallelism": f"replicas x{world}",
                        "l2": f"inputs rotated over {res['copies']} copies (> L2) between steps",
                        "timing": "CUDA graph replay per step"},
             "roofline": res["roofline"], "step_roofline": res["step_roofline"],

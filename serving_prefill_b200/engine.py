@@ -45,12 +45,15 @@ class PrefillEngine:
     def select(self):
         rag_impact_topk(self.impact, self.batch, self.r, self.k_cap, self.topk_idx, self.topk_val, self.k)
 
-    def step(self, layers, impact_layer: int, outs=None):
-        """layers: list of (layer index, q, kq, vq). outs: optional per-layer O buffers."""
+    def step(self, layers, impact_layer, outs=None):
+        """layers: list of (layer index, q, kq, vq). outs: optional per-layer O buffers.
+        impact_layer: the layer that feeds Impact and the top-k, or None (decode:
+        attention only)."""
         for n, (layer, q, kq, vq) in enumerate(layers):
             self.attend(layer, q, kq, vq, with_impact=(layer == impact_layer),
                         o=None if outs is None else outs[n])
-        self.select()
+        if impact_layer is not None:
+            self.select()
 
     def device_error(self):
         return rag_last_device_error(self.ws)

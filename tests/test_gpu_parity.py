@@ -34,6 +34,8 @@ def small_cases():
         "pooled": scaled(b16, num_q_heads=8, num_kv_heads=2, n_requests=5, n_pool_chunks=12,
                          chunk_len_range=(1, 400), chunks_per_req=(1, 4), q_range=(1, 90)),
         "g8_long_rows": scaled(l70, num_q_heads=16, num_kv_heads=2, chunk_lens=(700,) * 6, q_len=150),
+        "decode": scaled(get_workload("decode16"), num_q_heads=8, num_kv_heads=2, n_requests=6, n_pool_chunks=10,
+                         chunk_len_range=(1, 300), chunks_per_req=(1, 4), context_range=(1, 200)),
         "one_query_token": scaled(l2, num_q_heads=8, num_kv_heads=8, chunk_lens=(1, 15, 16, 17, 129), q_len=1),
         "query_longer_than_tile": scaled(l3, num_layers=1, num_q_heads=4, num_kv_heads=2, chunk_lens=(60,),
                                          q_len=300),
@@ -132,6 +134,14 @@ def test_parity_full_size(name):
     w = get_workload(name)
     case = DeviceCase(w, layers=[w.impact_layer_index])
     check_layer(case, w.impact_layer_index, with_impact=True)
+
+
+@pytest.mark.slow
+def test_parity_full_size_decode():
+    """One decode step of 16 requests: a new token over retrieved chunks and the request's own context."""
+    w = get_workload("decode16")
+    case = DeviceCase(w, layers=[0])
+    check_layer(case, 0, with_impact=False)
 
 
 @pytest.mark.slow

@@ -51,6 +51,11 @@ class Workload:
     chunk_len_range: tuple = (0, 0)
     chunks_per_req: tuple = (0, 0)
     q_range: tuple = (0, 0)
+    # decode steps: every request also holds a private chunk (its prompt and the
+    # tokens generated so far) of a length drawn from this range, after its
+    # retrieved chunks; the query block is the one new token
+    context_range: tuple = (0, 0)
+    select: bool = True             # run Impact and the top-k (prefill) or not (decode)
 
     @property
     def group(self) -> int:
@@ -65,7 +70,10 @@ class Workload:
         return 2 if self.dtype == "bf16" else 4
 
     @property
-    def impact_layer_index(self) -> int:
+    def impact_layer_index(self):
+        """The layer whose attention feeds Impact and the top-k; None for decode."""
+        if not self.select:
+            return None
         return self.num_layers - 1 if self.impact_layer < 0 else self.impact_layer
 
 
@@ -91,6 +99,14 @@ WORKLOADS = {
         head_dim=128, dtype="bf16", r=0.1, seed=1003, kind="pooled",
         n_requests=16, n_pool_chunks=256, chunk_len_range=(256, 1024),
         chunks_per_req=(4, 8), q_range=(32, 128)),
+    # decode over the fused cache: the batched16 requests one generation step
+    # later; each holds its prompt (32-128 tokens) and up to 256 generated
+    # tokens as a private chunk and attends with one new token
+    "decode16": Workload(
+        name="decode16", num_layers=1, num_q_heads=32, num_kv_heads=8,
+        head_dim=128, dtype="bf16", r=0.1, seed=1005, kind="pooled",
+        n_requests=16, n_pool_chunks=256, chunk_len_range=(256, 1024),
+        chunks_per_req=(4, 8), q_range=(1, 1), context_range=(33, 384), select=False),
     # 70B-shaped single layer, 64q/8kv, 32 x 2048 + 256 query, 4 outliers
     "long70b": Workload(
         name="long70b", num_layers=1, num_q_heads=64, num_kv_heads=8,
@@ -222,6 +238,10 @@ def make_layout(w: Workload) -> BatchLayout:
             n = int(torch.randint(w.chunks_per_req[0], w.chunks_per_req[1] + 1, (1,), generator=g))
             req_chunks.append(torch.randint(0, w.n_pool_chunks, (n,), generator=g).tolist())
             q_lens.append(int(torch.randint(w.q_range[0], w.q_range[1] + 1, (1,), generator=g)))
+        if w.context_range[1] > 0:
+            for cs in req_chunks:
+                cs.append(len(chunk_len))
+                chunk_len.append(int(torch.randint(w.context_range[0], w.context_range[1] + 1, (1,), generator=g)))
     n_pages = [-(-n // PAGE_SIZE) for n in chunk_len]
     num_pages = sum(n_pages)
     perm = torch.randperm(num_pages, generator=g)
