@@ -36,6 +36,11 @@ def small_cases():
         "g8_long_rows": scaled(l70, num_q_heads=16, num_kv_heads=2, chunk_lens=(700,) * 6, q_len=150),
         "decode": scaled(get_workload("decode16"), num_q_heads=8, num_kv_heads=2, n_requests=6, n_pool_chunks=10,
                          chunk_len_range=(1, 300), chunks_per_req=(1, 4), context_range=(1, 200)),
+        "decode_mha": scaled(get_workload("decode16"), num_q_heads=4, num_kv_heads=4, n_requests=3, n_pool_chunks=6,
+                             chunk_len_range=(1, 700), chunks_per_req=(1, 3), context_range=(1, 64)),
+        "decode_g8_long": scaled(get_workload("decode16"), num_q_heads=16, num_kv_heads=2, n_requests=2,
+                                 n_pool_chunks=4, chunk_len_range=(2000, 5000), chunks_per_req=(3, 4),
+                                 context_range=(300, 400)),
         "one_query_token": scaled(l2, num_q_heads=8, num_kv_heads=8, chunk_lens=(1, 15, 16, 17, 129), q_len=1),
         "query_longer_than_tile": scaled(l3, num_layers=1, num_q_heads=4, num_kv_heads=2, chunk_lens=(60,),
                                          q_len=300),
