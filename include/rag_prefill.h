@@ -63,7 +63,7 @@ typedef enum {
   RAG_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad scalar            */
   RAG_ERR_SHAPE = 2,       /* inconsistent sizes                              */
   RAG_ERR_PAGE_OOB = 3,    /* device: a page id outside [0, num_pages)        */
-  RAG_ERR_UNSUPPORTED = 4, /* valid request this build does not implement      */
+  RAG_ERR_UNSUPPORTED = 4, /* valid request the library does not implement    */
   RAG_ERR_CUDA = 5,        /* a CUDA runtime call failed                      */
   RAG_ERR_TIMEOUT = 6,     /* device: a pipeline wait gave up                 */
   RAG_ERR_WORKSPACE = 7,   /* workspace missing or smaller than required      */

@@ -8,4 +8,4 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
-    config.addinivalue_line("markers", "slow: full-size workload on the GPU box")
+    config.addinivalue_line("markers", "slow: full-size workload on a B200")
