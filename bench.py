@@ -289,12 +289,9 @@ def run_gpu(args, w, rank, world, device):
     del prof_graph
     clk = clocks.stop()
 
-    t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, device)
     ms_per_step = ms_max / args.steps
-    value = world * work["doc_tokens"] * args.steps / (ms_max / 1e3)
+    value = whole_job_rate(world, work["doc_tokens"], args.steps, ms_max)
 
     # dominant kernel and its roofline
     peaks = load_peaks()
@@ -384,13 +381,9 @@ def run_e2e(args, w, lay, layer_inputs, rep, device, world):
         one()
     ev1.record()
     torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
     doc = sum(lay.doc_lens)
-    return {"value": world * doc * steps / (ms / 1e3), "unit": "doc-KV tokens/s", "h2d_bytes_per_step": h2d,
+    return {"value": whole_job_rate(world, doc, steps, ms), "unit": "doc-KV tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps}
 
 
@@ -485,6 +478,21 @@ def run_reference(args, w, budget_per_step=None):
               f"heads) of every layer: pool write, gather, {what}; "
               f"tokens/s scaled by the group fraction")
     return value, dt / args.steps, sample
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def max_over_ranks(ms: float, world: int, device="cpu") -> float:
+    """The slowest rank's time: every rank takes part in one MAX reduction."""
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank_step: float, steps: int, ms_max: float) -> float:
+    """Units every rank processed in `steps` steps, over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (ms_max / 1e3)
 
 
 # ----------------------------------------------------------------------------- main
