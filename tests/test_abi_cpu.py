@@ -84,6 +84,9 @@ def test_validation_rejects_before_launch():
     bad = fake_batch()
     bad.max_q = 1000                                           # max above total
     assert attn(pool, bad) == 2
+    many = fake_batch()
+    many.num_requests = 4097                                   # above the 4,096 requests a batch may hold
+    assert attn(pool, many) == 4
 
 
 def test_pool_write_validation():

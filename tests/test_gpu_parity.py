@@ -142,6 +142,15 @@ def test_parity_full_size(name):
 
 
 @pytest.mark.slow
+def test_parity_at_the_request_limit():
+    """4,096 small requests, the most a batch may hold: prefixes, grids and the per-request top-k at full width."""
+    w = scaled(get_workload("batched16"), name="requests_4096", num_q_heads=4, num_kv_heads=2, n_requests=4096,
+               n_pool_chunks=64, chunk_len_range=(1, 40), chunks_per_req=(1, 2), q_range=(1, 3))
+    case = DeviceCase(w, layers=[0])
+    check_layer(case, 0, with_impact=True)
+
+
+@pytest.mark.slow
 def test_parity_full_size_decode():
     """One decode step of 16 requests: a new token over retrieved chunks and the request's own context."""
     w = get_workload("decode16")
