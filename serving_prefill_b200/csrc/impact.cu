@@ -11,8 +11,15 @@
 //
 //   producer warp : Q rows of the block (TMA, once per item) and K tiles
 //                   gathered through the page table (TMA page boxes)
-//   MMA warp      : S^T (128 keys x N rows) = K (smem) x Q^T (smem) -> TMEM
-//   4 epilogue warps: exp2 / scale / accumulate per key, atomicAdd
+//   MMA warp      : S^T (128 keys x N rows) = K (smem) x Q^T (smem) -> TMEM,
+//                   two S buffers ahead of the epilogue
+//   8 epilogue warps: two per TMEM lane quarter, each over half of the rows;
+//                   per key 2^(s c + b_row), with the row's normaliser folded
+//                   into the bias b_row = log2(1 / (l H_q)) - m2, summed on
+//                   MUFU exp2, the halves added in shared memory, atomicAdd
+// The producer and MMA warps start while the kernels before this one finish
+// (programmatic dependent launch); the epilogue waits for their row
+// statistics.
 // Impact is averaged over the H_q query heads (1/H_q is folded into row_il),
 // so the impacts of all N_doc + q columns of a request add up to q.
 #include <cuda.h>
