@@ -56,7 +56,9 @@ struct FwdCtrl {
   uint64_t q_full, q_empty;
   uint64_t kfull[kKStages], kempty[kKStages];
   uint64_t vfull[kVStages], vempty[kVStages], vconv[kVStages];
-  uint64_t s_full[kQTiles], p_full[kQTiles], pv_done[kQTiles], o_free[kQTiles];
+  // s_full[b] / p_full[b]: S buffer b (Q tile b's columns; with one Q tile in
+  // the item, both buffers serve Q tile 0 in turn)
+  uint64_t s_full[kQTiles], p_full[kQTiles], pv_done[kQTiles], o_full[kQTiles], o_free[kQTiles];
   uint64_t teardown;
   uint64_t desc_full[kDescSlots], desc_empty[kDescSlots];
   TileDesc desc[kDescSlots];
@@ -166,6 +168,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(&ctl->s_full[q], 1);
       mbar_init(&ctl->p_full[q], 128);
       mbar_init(&ctl->pv_done[q], 1);
+      mbar_init(&ctl->o_full[q], 1);
       mbar_init(&ctl->o_free[q], 128);
     }
     mbar_init(&ctl->teardown, 1);
@@ -247,13 +250,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int qt = warp >> 2;
     const int r = tid & 127;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + col_s(qt);
     const uint32_t o_addr = tmem + lane_off + col_o(qt);
-    uint32_t t_glob = 0, n_s = 0;   // tiles seen by the CTA, S tiles processed on this Q tile
+    uint32_t t_glob = 0;            // tiles seen by the CTA
+    uint32_t n_sf0 = 0, n_sf1 = 0;  // completions of s_full[0] / s_full[1] consumed (one P written per completion)
+    uint32_t n_pvq = 0;             // PVs into O_qt issued before the current step
+    uint32_t n_of = 0;              // items whose O_qt has been read
     int bad = 0;
     for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
       const FwdItem it = decode_fwd_item(p, prefix, w);
       const int n = it.t_end - it.t_begin;
+      // One Q tile: warpgroup 0 alone, alternating between the two S buffers
+      // so that S of the next tile is computed during this tile's softmax.
+      const bool single = it.n_qt == 1;
       const bool active = qt < it.n_qt;
       const int pr = it.rb * kFwdRows + qt * kBM + r;
       const int tok = pr / G;
@@ -268,7 +276,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->desc_empty[slot]);
         if (!active) continue;
-        if (!mbar_wait(&ctl->s_full[qt], n_s & 1, abort_flag)) { bad = 1; break; }
+        const int sb = single ? (i & 1) : qt;   // S buffer of this step
+        const uint32_t s_addr = tmem + lane_off + col_s(sb);
+        if (!mbar_wait(&ctl->s_full[sb], (sb ? n_sf1 : n_sf0) & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
         float x[kBN];
         {
@@ -322,8 +332,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           need = true;
         }
         if (__any_sync(0xffffffffu, need)) {
-          // O must hold the previous tile's PV before it is rescaled
-          if (!mbar_wait(&ctl->pv_done[qt], (n_s - 1) & 1, abort_flag)) { bad = 1; break; }
+          // O must hold the previous tile's PV before it is rescaled. The PV
+          // before that is complete (it was issued ahead of this tile's QK,
+          // whose result is here), so the parity names exactly PV(n_pvq - 1).
+          if (!mbar_wait(&ctl->pv_done[qt], (n_pvq - 1) & 1, abort_flag)) { bad = 1; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -363,17 +375,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         l_sum += (ls01.x + ls01.y) + (ls23.x + ls23.y);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&ctl->p_full[qt]);
-        ++n_s;
+        mbar_arrive(&ctl->p_full[sb]);
+        if (sb) ++n_sf1; else ++n_sf0;
+        ++n_pvq;
       }
       if (bad) break;
       t_glob += n;
+      // completions of s_full[1] that the other warpgroup consumed: the odd
+      // tiles of a one-Q-tile item (warpgroup 0's), every tile of a two-Q-tile
+      // item (warpgroup 1's)
+      if (single && qt == 1) n_sf1 += uint32_t(n) / 2;
+      if (!single && qt == 0) n_sf1 += uint32_t(n);
       if (!active) continue;
 
       // ---- epilogue: O of this Q tile
       float o[kHeadDim];
       if (n > 0) {
-        if (!mbar_wait(&ctl->pv_done[qt], (n_s - 1) & 1, abort_flag)) { bad = 1; break; }
+        // the MMA warp commits o_full once per item after the item's last PV
+        if (!mbar_wait(&ctl->o_full[qt], n_of & 1, abort_flag)) { bad = 1; break; }
+        ++n_of;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -573,7 +593,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t idesc_pv = idesc_f16_f32(kBM, kHeadDim, 1);
       const uint32_t q_base = smem_u32(sQ);
       uint32_t t_glob = 0, q_iter = 0;
-      uint32_t n_pv[kQTiles] = {0, 0}, n_item[kQTiles] = {0, 0};   // PVs issued, items begun, per Q tile
+      uint32_t n_pf0 = 0, n_pf1 = 0;       // completions of p_full[0] / p_full[1] consumed
+      uint32_t n_item[kQTiles] = {0, 0};   // items begun, per Q tile
       int bad = 0;
       for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
         const FwdItem it = decode_fwd_item(p, prefix, w);
@@ -581,6 +602,53 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (n == 0) continue;
         if (!mbar_wait(&ctl->q_full, q_iter & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
+        if (it.n_qt == 1) {
+          // One Q tile, two S buffers: QK of tiles 0 and 1 first, then per tile
+          // i, PV(i) as soon as its P is written and QK(i + 2) into the buffer
+          // PV(i) has just read (issue order keeps them apart).
+          auto qk = [&](int j) {
+            const uint32_t t = t_glob + j;
+            const int s = t % kKStages;
+            if (!mbar_wait(&ctl->kfull[s], (t / kKStages) & 1, abort_flag)) return false;
+            const uint32_t k_base = smem_u32(sK + s * kTileBytes);
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kHeadDim / 16; ++kk)
+              mma_ss(tmem + col_s(j & 1), kmajor_desc(q_base, kk), kmajor_desc(k_base, kk), idesc_qk, kk > 0);
+            tc_commit(&ctl->s_full[j & 1]);
+            tc_commit(&ctl->kempty[s]);
+            if (j == n - 1) tc_commit(&ctl->q_empty);   // the rest of the item reads no Q
+            return true;
+          };
+          for (int j = 0; j < n && j < 2 && !bad; ++j)
+            if (!qk(j)) bad = 1;
+          for (int i = 0; i < n && !bad; ++i) {
+            const uint32_t t = t_glob + i;
+            const int sv = t % kVStages;
+            const int b = i & 1;
+            if (!mbar_wait(&ctl->vconv[sv], (t / kVStages) & 1, abort_flag)) { bad = 1; break; }
+            if (i == 0) {
+              if (n_item[0] > 0 && !mbar_wait(&ctl->o_free[0], (n_item[0] - 1) & 1, abort_flag)) { bad = 1; break; }
+              ++n_item[0];
+            }
+            uint32_t& npf = b ? n_pf1 : n_pf0;
+            if (!mbar_wait(&ctl->p_full[b], npf & 1, abort_flag)) { bad = 1; break; }
+            ++npf;
+            tc_fence_after();
+            const uint32_t v_base = smem_u32(sV + sv * kTileBytes);
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk)
+              mma_ts(tmem + col_o(0), tmem + col_s(b) + kk * 8, v_desc(v_base, kk), idesc_pv, (i > 0) || (kk > 0));
+            tc_commit(&ctl->pv_done[0]);
+            if (i == n - 1) tc_commit(&ctl->o_full[0]);
+            tc_commit(&ctl->vempty[sv]);
+            if (i + 2 < n && !qk(i + 2)) { bad = 1; break; }
+          }
+          if (bad) break;
+          t_glob += n;
+          ++q_iter;
+          continue;
+        }
         // Tensor-core order per step: PV_0(t-1), QK_0(t), PV_1(t-1), QK_1(t), so
         // that softmax 0 of tile t runs while the pipe does PV_1 and QK_1.
         for (int i = 0; i <= n && !bad; ++i) {
@@ -607,14 +675,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 ++n_item[q];
               }
-              if (!mbar_wait(&ctl->p_full[q], n_pv[q] & 1, abort_flag)) { bad = 1; break; }
+              uint32_t& npf = q ? n_pf1 : n_pf0;
+              if (!mbar_wait(&ctl->p_full[q], npf & 1, abort_flag)) { bad = 1; break; }
+              ++npf;
               tc_fence_after();
 #pragma unroll
               for (int kk = 0; kk < kBN / 16; ++kk)
                 mma_ts(tmem + col_o(q), tmem + col_s(q) + kk * 8, v_desc(v_base, kk), idesc_pv,
                        (i > 1) || (kk > 0));
               tc_commit(&ctl->pv_done[q]);
-              ++n_pv[q];
+              if (i == n) tc_commit(&ctl->o_full[q]);   // O_q of this item is complete
             }
             if (i < n) {
               // S_q = Q_q K^T for this tile. It overwrites P_q (aliased over S_q),
