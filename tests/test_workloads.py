@@ -53,3 +53,26 @@ def test_one_token_query_is_unmasked_attention_over_every_key():
             want = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=1.0 / np.sqrt(w.head_dim))
             np.testing.assert_allclose(res.o[q0, h], want[0, 0, 0].numpy(), rtol=1e-12, atol=1e-12)
         q0 += 1
+
+
+def test_roofline_numerators_match_the_counts_by_hand():
+    # bench.step_work feeds roofline.achieved; pin it to the counts worked out by
+    # hand from each workload's shape (one QK^T and one PV per visible pair,
+    # K and V of every doc token once per request)
+    import sys, os
+    sys.path.insert(0, os.path.abspath(os.path.join(os.path.dirname(__file__), "..")))
+    import bench
+    w = get_workload("llama2_7b_l1")
+    work = bench.step_work(w, make_layout(w))
+    pairs = 64 * 2048 + 64 * 65 // 2                      # doc keys for every row, causal inside the query
+    assert work["attn_flops_per_launch"] == 4 * 128 * 32 * pairs
+    assert abs(work["attn_flops_per_launch"] - 2.18e9) / 2.18e9 < 0.01
+    kv = 2 * 2048 * 32 * 128 * 2                           # K and V, bf16
+    assert abs(kv - 33.5e6) / 33.5e6 < 0.01
+    assert work["attn_bytes_per_launch"] == kv + 64 * (32 + 2 * 32) * 128 * 2 + 64 * 32 * 128 * 2
+    w70 = get_workload("long70b")
+    work70 = bench.step_work(w70, make_layout(w70))
+    pairs70 = 256 * 65536 + 256 * 257 // 2
+    assert work70["attn_flops_per_launch"] == 4 * 128 * 64 * pairs70
+    assert abs(work70["attn_flops_per_launch"] - 551e9) / 551e9 < 0.01
+    assert abs(2 * 65536 * 8 * 128 * 2 - 268e6) / 268e6 < 0.01
