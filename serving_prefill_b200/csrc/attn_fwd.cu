@@ -267,6 +267,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int tok = pr / G;
       const int head = it.g * G + (pr % G);
       const bool row_valid = active && tok < it.req.n_q;
+      // A warp whose 32 rows are all past the query block (short queries,
+      // decode steps) skips the softmax and the epilogue's loads and stores;
+      // it still waits for every S and O and makes every arrival, so the
+      // barrier phases stay in step with the warps that hold real rows.
+      const bool warp_live = __any_sync(0xffffffffu, row_valid);
       float m_ref = -INFINITY, l_sum = 0.f;
       for (int i = 0; i < n; ++i) {
         const uint32_t t = t_glob + i;
@@ -280,6 +285,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t s_addr = tmem + lane_off + col_s(sb);
         if (!mbar_wait(&ctl->s_full[sb], (sb ? n_sf1 : n_sf0) & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
+        if (!warp_live) {
+          mbar_arrive(&ctl->p_full[sb]);
+          if (sb) ++n_sf1; else ++n_sf0;
+          ++n_pvq;
+          continue;
+        }
         float x[kBN];
         {
           uint32_t u0[32], u1[32];
@@ -389,12 +400,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (!active) continue;
 
       // ---- epilogue: O of this Q tile
-      float o[kHeadDim];
       if (n > 0) {
         // the MMA warp commits o_full once per item after the item's last PV
         if (!mbar_wait(&ctl->o_full[qt], n_of & 1, abort_flag)) { bad = 1; break; }
         ++n_of;
         tc_fence_after();
+      }
+      if (!warp_live) {   // no row of this warp is read or written
+        if (n > 0) {
+          tc_fence_before();
+          mbar_arrive(&ctl->o_free[qt]);
+        }
+        continue;
+      }
+      float o[kHeadDim];
+      if (n > 0) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t u[32];
