@@ -14,7 +14,11 @@ inputs (pool, Q, K_q, V_q, workspace) that each step's working set has left
 the 126 MB L2 before it is touched again. Each copy's step is captured once
 in a CUDA graph and replayed.
 
-One JSON line is printed by rank 0. With --impl reference the same metric is
+One JSON line is printed by rank 0. The headline is the 32-layer
+Llama-3-8B-shaped workload; at one GPU the other workloads (one Llama-2-7B
+layer, 16 batched requests, the 70B-shaped long context, a decode step) are
+measured in the same run, each with its own roofline, end-to-end number and
+oracle baseline, under "per_config". With --impl reference the same metric is
 measured for the fp64 CPU oracle on the host cores (a bounded sample per step).
 """
 
@@ -39,7 +43,10 @@ import torch  # noqa: E402
 
 from workloads import get_workload, make_layer_inputs, make_layout  # noqa: E402
 
-DEFAULT_CONFIG = "llama2_7b_l1"
+DEFAULT_CONFIG = "llama3_8b_l32"
+# the other workloads, each measured in the same run and reported under
+# "per_config" of the one JSON line (single-GPU runs only)
+PER_CONFIG = ["llama2_7b_l1", "batched16", "long70b", "decode16"]
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "doc-KV tokens/s through fused attn+impact+top-k; % of roofline at 1 B200"
 
@@ -410,12 +417,13 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_step(w, lay, layer_inputs, groups):
-    """The oracle on a sample of KV-head groups of every layer, then top-k.
+def oracle_step(w, lay, layer_inputs, groups, layers=None):
+    """The oracle on a sample of KV-head groups of a sample of layers, then top-k.
 
     A group is one KV head with the G query heads that read it, so a sample
     of n groups is the same problem with n KV heads: its pool, gather and
-    attention all shrink in proportion.
+    attention all shrink in proportion. Layers are independent problems of
+    equal size; the selecting layer is always part of the sample.
     """
     import oracle.prefill as orc
     scale = 1.0 / np.sqrt(w.head_dim)
@@ -423,7 +431,7 @@ def oracle_step(w, lay, layer_inputs, groups):
     G = w.num_q_heads // w.num_kv_heads
     heads = [g * G + j for g in groups for j in range(G)]
     impact_all = None
-    for layer in range(w.num_layers):
+    for layer in (range(w.num_layers) if layers is None else layers):
         inp = layer_inputs[layer]
         pk = orc.new_pool(1, lay.num_pages, len(groups), w.head_dim, bits)
         pv = orc.new_pool(1, lay.num_pages, len(groups), w.head_dim, bits)
@@ -458,37 +466,46 @@ def run_reference(args, w, budget_per_step=None):
     lay = make_layout(w)
     layer_inputs = [make_layer_inputs(w, lay, layer) for layer in range(w.num_layers)]
     doc = sum(lay.doc_lens)
-    # Calibrate: double the number of KV-head groups (spread over the heads)
-    # while one step still fits the per-step budget; the oracle's cost per
-    # group depends on how many groups it holds, so it is measured, not
-    # extrapolated. When the whole workload fits, every group is timed.
+    # Calibrate: the sample is a set of layers (the selecting layer first) and
+    # of KV-head groups (spread over the heads). Double the layers, then the
+    # groups, while one step still fits the per-step budget; the oracle's cost
+    # per group depends on how many groups it holds, so it is measured, not
+    # extrapolated. When the whole workload fits, all of it is timed.
     budget = budget_per_step or max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    L = w.num_layers
+    first = w.impact_layer_index if w.impact_layer_index is not None else 0
 
-    def spread(n):
-        return list(range(0, w.num_kv_heads, max(1, w.num_kv_heads // n)))[:n]
+    def spread(n, total):
+        return list(range(0, total, max(1, total // n)))[:n]
 
-    n = 1
-    while n < w.num_kv_heads:
-        n2 = min(2 * n, w.num_kv_heads)
+    def layer_set(n):
+        rest = [x for x in spread(n, L) if x != first]
+        return sorted([first] + rest[: n - 1])
+
+    def fits(nl, ng):
         t0 = time.perf_counter()
-        oracle_step(w, lay, layer_inputs, spread(n2))
-        if time.perf_counter() - t0 > budget:
-            break
-        n = n2
-    groups = spread(n)
+        oracle_step(w, lay, layer_inputs, spread(ng, w.num_kv_heads), layer_set(nl))
+        return time.perf_counter() - t0 <= budget
+
+    nl, ng = 1, 1
+    while nl < L and fits(min(2 * nl, L), ng):
+        nl = min(2 * nl, L)
+    while nl == L and ng < w.num_kv_heads and fits(nl, min(2 * ng, w.num_kv_heads)):
+        ng = min(2 * ng, w.num_kv_heads)
+    groups, layers = spread(ng, w.num_kv_heads), layer_set(nl)
     for _ in range(args.warmup):
-        oracle_step(w, lay, layer_inputs, groups)
+        oracle_step(w, lay, layer_inputs, groups, layers)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(w, lay, layer_inputs, groups)
+        oracle_step(w, lay, layer_inputs, groups, layers)
     dt = time.perf_counter() - t0
-    frac = len(groups) / w.num_kv_heads
+    frac = len(groups) / w.num_kv_heads * len(layers) / L
     value = doc * frac * args.steps / dt
     G = w.num_q_heads // w.num_kv_heads
     what = "attention, impact, top-k over all doc tokens" if w.select else "attention (decode step)"
     sample = (f"{len(groups)} of {w.num_kv_heads} KV-head groups ({len(groups) * G} of {w.num_q_heads} query "
-              f"heads) of every layer: pool write, gather, {what}; "
-              f"tokens/s scaled by the group fraction")
+              f"heads) of {len(layers)} of {L} layers: pool write, gather, {what}; "
+              f"tokens/s scaled by the fraction of (layer, group) pairs timed")
     return value, dt / args.steps, sample
 
 
@@ -509,6 +526,24 @@ def whole_job_rate(world: int, units_per_rank_step: float, steps: int, ms_max: f
 
 # ----------------------------------------------------------------------------- main
 
+def cpu_baseline(w, budget_per_step):
+    """The oracle timed on the host cores over a bounded sample of the workload."""
+    small = argparse.Namespace(steps=2, warmup=1)
+    value, s_per_step, sample = run_reference(small, w, budget_per_step=budget_per_step)
+    return {"value": value, "unit": "doc-KV tokens/s" if w.select else "KV tokens/s", "cores": blas_threads(),
+            "kind": "oracle", "sample": sample + f"; 2 timed steps of {s_per_step:.2f} s"}
+
+
+def config_of(w, res, world):
+    lay = make_layout(w)
+    return {"workload": w.name, "requests": lay.num_requests, "layers": w.num_layers,
+            "doc_tokens_per_step": sum(lay.doc_lens), "query_tokens_per_step": lay.total_q,
+            "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+            "r": w.r if w.select else None, "parallelism": f"replicas x{world}",
+            "l2": f"inputs rotated over {res['copies']} copies (> L2) between steps",
+            "timing": "CUDA graph replay per step"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -517,6 +552,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="measure the headline workload only (no per_config block)")
     ap.add_argument("--ncu", action="store_true",
                     help="profiling mode: one input copy, eager launches, W + K steps, no JSON")
     args = ap.parse_args()
@@ -562,30 +599,36 @@ def main():
         sys.exit(0 if st == 0 else 1)
     res = run_gpu(args, w, rank, world, device)
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        small = argparse.Namespace(steps=2, warmup=1)
-        value, s_per_step, sample = run_reference(small, w, budget_per_step=5.0)
-        cpu = {"value": value, "unit": "doc-KV tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": sample + f"; 2 timed steps of {s_per_step:.2f} s"}
+    do_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    cpu = cpu_baseline(w, 5.0) if do_cpu else None
+
+    per_config = None
+    if world == 1 and not args.no_per_config and args.config == DEFAULT_CONFIG:
+        per_config = {}
+        for name in PER_CONFIG:
+            wc = get_workload(name)
+            rc = run_gpu(args, wc, rank, world, device)
+            torch.cuda.empty_cache()
+            entry = {"value": rc["value"], "unit": "doc-KV tokens/s" if wc.select else "KV tokens/s",
+                     "ms_per_step": rc["ms_per_step"], "config": config_of(wc, rc, world),
+                     "roofline": rc["roofline"], "step_roofline": rc["step_roofline"],
+                     "cpu_baseline": cpu_baseline(wc, 2.0) if do_cpu else None, "e2e": rc["e2e"],
+                     "gpu_launches": rc["gpu_launches"], "clocks": rc["clocks"], "kernels": rc["kernels"]}
+            per_config[name] = entry
 
     if rank == 0:
-        lay = make_layout(w)
         line = {
             "metric": METRIC, "value": res["value"], "unit": "doc-KV tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": {"workload": w.name, "requests": lay.num_requests, "layers": w.num_layers,
-                       "doc_tokens_per_step": sum(lay.doc_lens), "query_tokens_per_step": lay.total_q,
-                       "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
-                       "r": w.r if w.select else None, "parallelism": f"replicas x{world}",
-                       "l2": f"inputs rotated over {res['copies']} copies (> L2) between steps",
-                       "timing": "CUDA graph replay per step"},
+            "config": config_of(w, res, world),
             "roofline": res["roofline"], "step_roofline": res["step_roofline"],
             "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
             "clocks": res["clocks"], "kernels": res["kernels"], "kernel_timing": res["kernel_timing"],
         }
+        if per_config is not None:
+            line["per_config"] = per_config
         print(json.dumps(line))
     if world > 1:
         torch.distributed.barrier()

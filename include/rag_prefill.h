@@ -67,7 +67,10 @@ typedef enum {
   RAG_ERR_CUDA = 5,        /* a CUDA runtime call failed                      */
   RAG_ERR_TIMEOUT = 6,     /* device: a pipeline wait gave up                 */
   RAG_ERR_WORKSPACE = 7,   /* workspace missing or smaller than required      */
-  RAG_ERR_GEOMETRY = 8     /* device: chunk pages do not match its length     */
+  RAG_ERR_GEOMETRY = 8,    /* device: chunk pages do not match its length     */
+  RAG_ERR_RANGE = 9        /* device: a bf16 V value of magnitude >= 65536
+                              (or inf/nan) met the fp16 PV product and was
+                              saturated to +-65504; O is then inexact        */
 } rag_status;
 
 typedef enum { RAG_BF16 = 0, RAG_F32 = 1 } rag_dtype;
@@ -164,7 +167,12 @@ RAG_API rag_status rag_workspace_init(void* workspace, size_t workspace_bytes, v
  *   N_doc,b + q_b key positions i, (1/H_q) sum_h sum_j alpha^h_{j,i}; the doc
  *   part comes first. The impacts of a request's segment add up to q_b.
  *   Pass it on the layer whose attention selects tokens (the last layer).
- * workspace: device, >= rag_workspace_size() bytes, 256-byte aligned. */
+ * workspace: device, >= rag_workspace_size() bytes, 256-byte aligned.
+ * Precision (bf16 pool): scores and the softmax run in fp32; the PV product
+ * takes P and V in fp16, which holds every bf16 V value of magnitude up to
+ * 65280 (below 2^-14 with an absolute error under 2^-24). A V value of
+ * magnitude 65536 or more (or inf/nan) is saturated to +-65504 and the call
+ * reports RAG_ERR_RANGE through rag_last_device_error. */
 RAG_API rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch, const void* q,
                                   int32_t num_q_heads, const void* kq, const void* vq, float sm_scale, void* o,
                                   float* row_lse, float* impact, void* workspace, size_t workspace_bytes,
@@ -185,9 +193,14 @@ RAG_API rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer
  * (different streams, or different host threads, on one device) race on it;
  * serialise them on one stream.
  * The first call on each device looks up the array's device address (with that
- * device current); make that first call before any stream capture.
+ * device current); make that first call before any stream capture. The address
+ * is kept for the life of the process: after cudaDeviceReset (or any other
+ * reset of the device's primary context) the library's device image is loaded
+ * again and the kept address is stale, so a process that resets a device must
+ * not call this entry point on it afterwards.
  * device_err: optional device int32 that receives the call's device error bits
- * (as rag_last_device_error reports them: 1 page, 2 geometry, 4 timeout).
+ * (as rag_last_device_error reports them: 1 page, 2 geometry, 4 timeout,
+ * 8 range).
  * Other arguments and outputs as for rag_fused_prefill_attn. */
 RAG_API rag_status rag_fused_prefill_attn_static(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch,
                                                  const void* q, int32_t num_q_heads, const void* kq,
@@ -203,8 +216,10 @@ RAG_API int32_t rag_recompute_count(int32_t n_doc, double r);
  * `select_tokens_for_recompute`, torch.topk over the doc slice):
  * impact   as written by rag_fused_prefill_attn (device fp32)
  * r        recompute ratio, 0 < r < 1
- * k_cap    row length of the outputs, >= rag_recompute_count(max_doc, r),
- *          <= 8192
+ * k_cap    row length of the outputs, >= rag_recompute_count(max_doc, r).
+ *          The selection itself is limited to k = rag_recompute_count(max_doc,
+ *          r) <= 16384 per request (RAG_ERR_UNSUPPORTED above that); k_cap
+ *          may be larger, the rest of each row is padding
  * topk_idx [B][k_cap] int32 device output: the k_b doc positions of largest
  *          impact ordered by (impact descending, position ascending); the
  *          rest of the row is -1
@@ -215,9 +230,21 @@ RAG_API rag_status rag_impact_topk(const float* impact, const rag_batch* batch, 
 
 /* Synchronise `stream`, read and clear the workspace error word. Returns
  * RAG_OK when the device reported nothing, else the most severe of
- * RAG_ERR_TIMEOUT, RAG_ERR_PAGE_OOB, RAG_ERR_GEOMETRY; *bits (optional)
- * receives the raw bits (1 page, 2 geometry, 4 timeout). */
+ * RAG_ERR_TIMEOUT, RAG_ERR_PAGE_OOB, RAG_ERR_GEOMETRY, RAG_ERR_RANGE; *bits
+ * (optional) receives the raw bits (1 page, 2 geometry, 4 timeout, 8 range). */
 RAG_API rag_status rag_last_device_error(void* workspace, int32_t* bits, void* stream);
+
+/* Self-test of the device-side failure detection (not a step of the method;
+ * the pages have no counterpart). Launches one CTA on `stream` in which one
+ * role waits on an mbarrier that nothing completes, with a limit of limit_ns
+ * (1 .. 2e9 ns), while a second role waits on another such barrier with the
+ * pipelines' full 2 s limit. The first wait runs out, records the timeout bit
+ * (4) in *device_err (device int32, OR-ed in) and raises the CTA's abort flag;
+ * the second role must then leave at once. The kernel therefore ends after
+ * about limit_ns, never hangs, and leaves the context usable: this is the
+ * mechanism every pipeline wait of the library uses to turn a stall into
+ * RAG_ERR_TIMEOUT. */
+RAG_API rag_status rag_selftest_wait_timeout(int32_t* device_err, int64_t limit_ns, void* stream);
 
 /* Kernel launches this library has made in this process (all entry points). */
 RAG_API int64_t rag_launch_count(void);

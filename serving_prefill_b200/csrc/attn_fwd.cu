@@ -577,10 +577,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   } else if (warp == 11) {
     // ------------------------------------------------------------ V converter
     // The PV product runs in fp16 (P and V): P keeps 3 more mantissa bits than
-    // bf16, and every bf16 V value of magnitude in [2^-14, 65504] is exact in
-    // fp16. The tile is rewritten in place; the 128B swizzle is unchanged.
+    // bf16, and every bf16 V value of magnitude in [2^-14, 65280] is exact in
+    // fp16 (smaller ones keep an absolute error below 2^-24). Magnitudes from
+    // 65536 up (and inf, nan) do not fit: they saturate, and the tile raises
+    // kDevErrRange. The tile is rewritten in place; the 128B swizzle is
+    // unchanged.
     uint32_t t_glob = 0;
     int bad = 0;
+    uint32_t range = 0;   // bit 15 of a halfword: some |v| >= 65536 (bf16 0x4780)
     for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
       const FwdItem it = decode_fwd_item(p, prefix, w);
       const int n = it.t_end - it.t_begin;
@@ -592,6 +596,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll 4
         for (int v = lane; v < kTileBytes / 16; v += 32) {
           uint4 x = tile[v];
+          // |h| + 0x3880 reaches 0x8000 exactly when |h| >= 0x4780; no carry
+          // crosses into the other halfword
+          range |= ((x.x & 0x7fff7fffu) + 0x38803880u) | ((x.y & 0x7fff7fffu) + 0x38803880u) |
+                   ((x.z & 0x7fff7fffu) + 0x38803880u) | ((x.w & 0x7fff7fffu) + 0x38803880u);
           x.x = bf16x2_to_f16x2(x.x);
           x.y = bf16x2_to_f16x2(x.y);
           x.z = bf16x2_to_f16x2(x.z);
@@ -605,6 +613,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       t_glob += n;
     }
     if (bad) raise_abort(ctl, p.err);
+    if (__any_sync(0xffffffffu, (range & 0x80008000u) != 0) && lane == 0) atomicOr(p.err, kDevErrRange);
     __syncwarp();
   } else {
     // ------------------------------------------------------------ MMA issuer (warp 10)
@@ -835,12 +844,9 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const CUtensorMap& tkq, const CUtensorMap& tvq, const FwdParams& p, int grid,
                             cudaStream_t stream) {
   const size_t smem = fwd_smem_bytes(p.batch.num_requests);
-  static size_t attr_set = 0;   // largest dynamic smem size configured so far
-  if (smem > attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = smem;
-  }
+  static SmemAttr attr;
+  cudaError_t e = ensure_smem_attr(attn_fwd_kernel, attr, smem);
+  if (e != cudaSuccess) return e;
   return launch_pdl(attn_fwd_kernel, dim3(grid), dim3(kFwdThreads), smem, stream, 1, tq, tk, tv, tkq, tvq, p);
 }
 

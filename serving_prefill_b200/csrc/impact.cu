@@ -412,12 +412,9 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 cudaError_t launch_impact(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tkq,
                           const ImpactParams& p, int grid, cudaStream_t stream) {
   const size_t smem = impact_smem_bytes(p.batch.num_requests);
-  static size_t attr_set = 0;   // largest dynamic smem size configured so far
-  if (smem > attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(impact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = smem;
-  }
+  static SmemAttr attr;
+  cudaError_t e = ensure_smem_attr(impact_kernel, attr, smem);
+  if (e != cudaSuccess) return e;
   return launch_pdl(impact_kernel, dim3(grid), dim3(kImpThreads), smem, stream, 1, tq, tk, tkq, p);
 }
 

@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
 #include <utility>
 
 #include "common.cuh"
@@ -39,6 +40,29 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
+// cudaFuncSetAttribute acts on the current device's context only, so the
+// largest dynamic shared-memory size set for a kernel is kept per device (and
+// the record is shared by host threads under a mutex).
+constexpr int kMaxDevices = 64;
+struct SmemAttr {
+  std::mutex mu;
+  size_t bytes[kMaxDevices] = {};
+};
+template <typename Kernel>
+inline cudaError_t ensure_smem_attr(Kernel kernel, SmemAttr& rec, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(rec.mu);
+  if (bytes > rec.bytes[dev]) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+    if (e != cudaSuccess) return e;
+    rec.bytes[dev] = bytes;
+  }
+  return cudaSuccess;
+}
+
 struct FwdParams {
   BatchDev batch;
   int32_t num_pages, num_kv_heads, num_q_heads, group, layer;

@@ -18,7 +18,7 @@
 namespace rag {
 
 constexpr int kSimtMaxKeysHost = 8192;
-constexpr int kTopkMaxKHost = 8192;
+constexpr int kTopkMaxKHost = 16384;
 
 // ------------------------------------------------------------ profiling
 
@@ -242,6 +242,7 @@ const char* rag_status_string(int32_t s) {
     case RAG_ERR_TIMEOUT: return "device pipeline wait timed out";
     case RAG_ERR_WORKSPACE: return "workspace missing or too small";
     case RAG_ERR_GEOMETRY: return "chunk page count does not match its length";
+    case RAG_ERR_RANGE: return "a V value beyond the fp16 range was saturated";
     default: return "unknown status";
   }
 }
@@ -500,6 +501,7 @@ rag_status rag_last_device_error(void* workspace, int32_t* bits, void* stream) {
   if (host & kDevErrTimeout) return RAG_ERR_TIMEOUT;
   if (host & kDevErrPage) return RAG_ERR_PAGE_OOB;
   if (host & kDevErrGeometry) return RAG_ERR_GEOMETRY;
+  if (host & kDevErrRange) return RAG_ERR_RANGE;
   return RAG_OK;
 }
 

@@ -162,12 +162,9 @@ __global__ void __launch_bounds__(kSimtThreads) simt_impact_kernel(const SimtPar
 
 cudaError_t launch_simt_attn(const SimtParams& p, int total_q, cudaStream_t stream) {
   const size_t smem = sizeof(float) * (p.head_dim + kSimtMaxKeys) + sizeof(int64_t) * kSimtMaxKeys;
-  static size_t attr_set = 0;   // largest dynamic smem size configured so far
-  if (smem > attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(simt_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = smem;
-  }
+  static SmemAttr attr;
+  cudaError_t e = ensure_smem_attr(simt_attn_kernel, attr, smem);
+  if (e != cudaSuccess) return e;
   simt_attn_kernel<<<dim3(total_q, p.num_q_heads), kSimtThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }

@@ -12,9 +12,10 @@
 // ascending) of its keys above d1, and of the candidates inside d1, into CTA
 // 0's shared memory, bucket by bucket. CTA 0 sorts every bucket on its own
 // (a warp per bucket, the whole CTA for a bucket of more than 1,024 keys);
-// the first k keys are then the answer in order. When d1 holds more keys than
-// fit, CTA 0 finds the k-th key by an exact radix select on the remaining 20
-// bits instead and sorts the k keys.
+// the first k keys are then the answer in order. When the keys above d1 and
+// d1's candidates together exceed the 20,480 that shared memory stages, CTA 0
+// finds the k-th key by an exact radix select on the remaining 20 bits
+// instead and sorts the k keys. k is at most 16,384.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
@@ -28,9 +29,8 @@ constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkBins = 4096;
 constexpr int kBatch = 8;            // keys in flight per thread per pass
-constexpr int kTopkMaxK = 8192;      // largest k
-constexpr int kTopkCand = 8192;      // candidates of the k-th key's bucket staged in shared memory
-constexpr int kTopkSortMax = kTopkMaxK + kTopkCand;   // staged keys
+constexpr int kTopkMaxK = 16384;     // largest k
+constexpr int kTopkSortMax = 20480;  // staged keys: those above the k-th key's bucket, then its candidates
 constexpr int kTopkMaxCluster = 8;
 constexpr int kTopkSlice = 8192;     // doc tokens per CTA before the cluster grows
 constexpr int kRankMax = 256;        // longest bucket ordered by counting ranks (longer: sorted)
@@ -269,10 +269,36 @@ __device__ void block_sort(uint64_t* a, int len) {
   __syncthreads();
 }
 
+// The same network with every step in shared memory (runs longer than the
+// register forms hold: more than 8,192 keys).
+__device__ void block_sort_smem(uint64_t* a, int len) {
+  const int tid = threadIdx.x;
+  int sp = 2;
+  while (sp < len) sp <<= 1;
+  __syncthreads();
+  for (int size = 2; size <= sp; size <<= 1) {
+    const int half = size >> 1, lg_half = __ffs(half) - 1;
+    for (int q = tid; q < (sp >> 1); q += kTopkThreads) {
+      const int base = (q >> lg_half) * size, off = q & (half - 1);
+      const int i = base + off, j = base + size - 1 - off;
+      if (j < len) cmpswap(a[i], a[j]);
+    }
+    __syncthreads();
+    for (int st = size >> 2; st >= 1; st >>= 1) {
+      for (int q = tid; q < (sp >> 1); q += kTopkThreads) {
+        const int i = 2 * q - (q & (st - 1)), j = i + st;
+        if (j < len) cmpswap(a[i], a[j]);
+      }
+      __syncthreads();
+    }
+  }
+}
+
 __device__ void block_sort_any(uint64_t* a, int len) {
   if (len <= 64 * kTopkWarps) block_sort<2>(a, len);
   else if (len <= 128 * kTopkWarps) block_sort<4>(a, len);
-  else block_sort<8>(a, len);
+  else if (len <= 256 * kTopkWarps) block_sort<8>(a, len);
+  else block_sort_smem(a, len);
 }
 
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams p) {
@@ -328,7 +354,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   const int kr1 = int(S.sel[1]);
   const int n_gt1 = k - kr1;
   const int nc = int(S.ghist[d1]);
-  const bool stage_cand = nc <= kTopkCand;
+  const bool stage_cand = n_gt1 + nc <= kTopkSortMax;
   // Staging: the keys of the buckets above d1 in descending bucket order, then
   // the candidates. Every bucket from d1 up that holds keys is a segment;
   // segment g (in descending bucket order) is ordered by CTA g % C, and only
@@ -537,12 +563,9 @@ int topk_cluster_size(int max_doc) {
 cudaError_t launch_topk(const TopkParams& p, int num_requests, int max_k, cudaStream_t stream) {
   (void)max_k;
   const size_t smem = topk_smem_bytes();
-  static size_t attr_set = 0;   // largest dynamic smem size configured so far
-  if (smem > attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = smem;
-  }
+  static SmemAttr attr;
+  cudaError_t e = ensure_smem_attr(topk_kernel, attr, smem);
+  if (e != cudaSuccess) return e;
   const int c = topk_cluster_size(p.batch.max_doc);
   return launch_pdl(topk_kernel, dim3(num_requests * c), dim3(kTopkThreads), smem, stream, c, p);
 }

@@ -24,6 +24,7 @@ STATUS = {
     0: "ok", 1: "invalid argument", 2: "inconsistent shape", 3: "page id outside the pool",
     4: "unsupported configuration", 5: "CUDA runtime error", 6: "device pipeline wait timed out",
     7: "workspace missing or too small", 8: "chunk page count does not match its length",
+    9: "a V value beyond the fp16 range was saturated",
 }
 
 
@@ -65,6 +66,7 @@ EXPORTS = {
     "rag_impact_topk": (c_int32, [c_void_p, POINTER(RagBatch), c_double, c_int32, c_void_p, c_void_p, c_void_p,
                                   c_void_p]),
     "rag_last_device_error": (c_int32, [c_void_p, c_void_p, c_void_p]),
+    "rag_selftest_wait_timeout": (c_int32, [c_void_p, c_int64, c_void_p]),
     "rag_launch_count": (c_int64, []),
     "rag_profile_enable": (None, [c_int32]),
     "rag_profile_collect": (c_int32, [c_void_p, c_void_p, c_int32]),
@@ -222,6 +224,11 @@ def rag_last_device_error(workspace: torch.Tensor, stream=None) -> tuple:
     bits = c_int32(0)
     st = lib().rag_last_device_error(_ptr(workspace), ctypes.byref(bits), _stream(stream))
     return st, bits.value
+
+
+def rag_selftest_wait_timeout(device_err: torch.Tensor, limit_ns: int, stream=None):
+    _check(lib().rag_selftest_wait_timeout(_ptr(device_err), limit_ns, _stream(stream)),
+           "rag_selftest_wait_timeout")
 
 
 def rag_launch_count() -> int:

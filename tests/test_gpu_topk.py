@@ -93,3 +93,30 @@ def test_large_buckets_use_wide_sorts():
 def test_many_buckets_across_the_cluster():
     rng = np.random.default_rng(8)
     check([rng.lognormal(-6, 2.5, 65536)], 0.1)   # hundreds of buckets dealt over eight CTAs
+
+
+def test_k_above_eight_thousand():
+    # 65,536 doc tokens at r = 0.15, inside the pages' 0.05-0.15 range: k = 9,830
+    rng = np.random.default_rng(9)
+    check([rng.lognormal(-6, 1.0, 65536)], 0.15)
+    check([rng.random(65536), rng.random(300)], 0.15)
+
+
+def test_k_at_the_limit():
+    # k = int(109,227 * 0.15) = 16,384, the largest selection a request may make
+    rng = np.random.default_rng(10)
+    n = 109227
+    assert rag_recompute_count(n, 0.15) == 16384
+    check([rng.lognormal(-5, 1.2, n)], 0.15)
+
+
+def test_bucket_above_the_kth_longer_than_a_register_sort():
+    # 10,000 keys in one 12-bit bucket above the k-th key's bucket: that segment
+    # is longer than the 8,192 keys the register sorting networks hold
+    rng = np.random.default_rng(11)
+    a = 2.0 + 0.25 * rng.random(10000)        # [2, 2.25): one bucket
+    b = 1.0 + 0.125 * rng.random(10000)       # [1, 1.125): the bucket below it
+    low = 0.5 * rng.random(80000)
+    seg = np.concatenate([low[:40000], a, low[40000:], b])
+    n = len(seg)
+    check([seg], 12000.5 / n)                  # k = 12,000: all of a, 2,000 of b
