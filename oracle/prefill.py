@@ -173,7 +173,13 @@ def attend_request(q: np.ndarray, kcat: np.ndarray, vcat: np.ndarray, n_doc: int
 # --------------------------------------------------------------------------
 
 def recompute_count(n_doc: int, r: float) -> int:
-    """k = max(1, int(N_doc * r)), with the product taken in double precision."""
+    """k = max(1, int(N_doc * r)), with the product taken in double precision.
+
+    A request with no doc tokens has nothing to select: k = 0 (the listing's
+    max(1, .) is read as applying to a non-empty doc slice).
+    """
+    if n_doc <= 0:
+        return 0
     return max(1, int(n_doc * r))
 
 

@@ -278,6 +278,14 @@ def test_recompute_count_golden():
         assert orc.recompute_count(c["n_doc"], float(c["r"])) == c["k"], c
 
 
+def test_recompute_count_of_an_empty_doc_slice_is_zero():
+    """A request with no doc tokens has nothing to select (the max(1, .) floor
+    applies to a non-empty slice); the selection of such a request is empty."""
+    for r in (0.05, 0.1, 0.15, 0.99):
+        assert orc.recompute_count(0, r) == 0
+        assert orc.select_topk(np.zeros(0), orc.recompute_count(0, r)).tolist() == []
+
+
 @pytest.mark.parametrize("r", ["0.05", "0.1", "0.15"])
 def test_recompute_count_is_exact_floor(r):
     """int(N * r) in double equals floor(N * r) over the exact decimal r."""
