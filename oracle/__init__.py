@@ -15,3 +15,4 @@ from .prefill import (  # noqa: F401
     run_workload,
     OracleResult,
 )
+from . import recompute  # noqa: F401

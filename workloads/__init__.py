@@ -12,6 +12,8 @@ from .rag import (  # noqa: F401
     Workload,
     BatchLayout,
     LayerInputs,
+    RecomputeInputs,
+    make_recompute_inputs,
     make_layout,
     make_layer_inputs,
     get_workload,

@@ -56,6 +56,7 @@ class Workload:
     # retrieved chunks; the query block is the one new token
     context_range: tuple = (0, 0)
     select: bool = True             # run Impact and the top-k (prefill) or not (decode)
+    d_model: int = 4096             # hidden size feeding the K/V projections (selective recompute)
 
     @property
     def group(self) -> int:
@@ -111,7 +112,7 @@ WORKLOADS = {
     "long70b": Workload(
         name="long70b", num_layers=1, num_q_heads=64, num_kv_heads=8,
         head_dim=128, dtype="bf16", r=0.05, seed=1004, n_outliers=4,
-        chunk_lens=(2048,) * 32, q_len=256),
+        chunk_lens=(2048,) * 32, q_len=256, d_model=8192),
 }
 
 # index order of the workloads as the headline configuration list gives them
@@ -141,7 +142,7 @@ def _gen(seed: int, *tags: int) -> torch.Generator:
 
 
 # sub-stream tags
-_T_LAYOUT, _T_SCALE, _T_Q, _T_K, _T_V, _T_KQ, _T_VQ = range(7)
+_T_LAYOUT, _T_SCALE, _T_Q, _T_K, _T_V, _T_KQ, _T_VQ, _T_X, _T_WK, _T_WV = range(10)
 
 
 @dataclass
@@ -294,3 +295,26 @@ def make_layer_inputs(w: Workload, lay: BatchLayout, layer: int) -> LayerInputs:
     kq = (torch.randn(tq, hk, d, generator=_gen(w.seed, _T_KQ, layer)) * sk).to(dt)
     vq = (torch.randn(tq, hk, d, generator=_gen(w.seed, _T_VQ, layer)) * sv).to(dt)
     return LayerInputs(chunk_k=ck, chunk_v=cv, q=q, kq=kq, vq=vq)
+
+
+@dataclass
+class RecomputeInputs:
+    """One layer's inputs of the selective recompute.
+
+    x: hidden states of the batch's doc tokens [total_doc, d_model] (request
+    order, then position), N(0, 1); w_k, w_v: projection weights
+    [H_kv * head_dim, d_model] (a linear layer's layout), N(0, 1 / d_model), so
+    that a projected value is about N(0, 1); all rounded once to bf16.
+    """
+    x: torch.Tensor
+    w_k: torch.Tensor
+    w_v: torch.Tensor
+
+
+def make_recompute_inputs(w: Workload, lay: BatchLayout, layer: int) -> RecomputeInputs:
+    n_out = w.num_kv_heads * w.head_dim
+    std = 1.0 / float(w.d_model) ** 0.5
+    x = torch.randn(lay.total_doc, w.d_model, generator=_gen(w.seed, _T_X, layer)).to(torch.bfloat16)
+    wk = (torch.randn(n_out, w.d_model, generator=_gen(w.seed, _T_WK, layer)) * std).to(torch.bfloat16)
+    wv = (torch.randn(n_out, w.d_model, generator=_gen(w.seed, _T_WV, layer)) * std).to(torch.bfloat16)
+    return RecomputeInputs(x=x, w_k=wk, w_v=wv)
