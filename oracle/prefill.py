@@ -118,6 +118,56 @@ def gather(pool: np.ndarray, layer: int, chunks) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# step 2b (optional): RoPE position re-basing of the cached keys
+# --------------------------------------------------------------------------
+#
+# TurboRAG page, "Implementation": with rotary position embeddings, the
+# position ids used when a chunk's cache is precomputed and those used at
+# inference must agree. A chunk precomputed on its own carries RoPE at its
+# local positions 0 .. n_c - 1; in the concatenated sequence it starts at
+# offset o (the doc tokens of the chunks before it). Re-basing rotates every
+# cached key by the angle o * theta_i of its rotary pair, which moves it to
+# position o + t (rotations of one pair add their angles). Convention (Llama's
+# rotary embedding): pair i couples channels i and i + d/2, theta_i =
+# base^(-2 i / d). The re-based key is held in the cache dtype: the rotation
+# is exact (fp64) and the result is rounded once to bf16.
+
+def rope_theta_i(head_dim: int, base: float) -> np.ndarray:
+    """Angle per position of each rotary pair: base^(-2 i / d), i < d / 2."""
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    return np.power(float(base), -2.0 * i / head_dim)
+
+
+def rope_rotate(k: np.ndarray, offset: int, base: float) -> np.ndarray:
+    """Rotate keys [..., d] (fp64) by offset positions: pair (i, i + d/2) turns
+    by offset * theta_i."""
+    d = k.shape[-1]
+    ang = float(offset) * rope_theta_i(d, base)
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = k[..., : d // 2], k[..., d // 2:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def rope_rebase_bits(k_bits: np.ndarray, offset: int, base: float) -> np.ndarray:
+    """Re-based cached keys in the cache dtype (bf16 bits), rounded once."""
+    r = rope_rotate(bits_to_f64(k_bits), offset, base)
+    t = torch.from_numpy(np.ascontiguousarray(r)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def gather_rebased(pool: np.ndarray, layer: int, chunks, base: float) -> np.ndarray:
+    """gather() with every chunk's keys re-based to its offset in the request."""
+    parts, at = [], 0
+    for page_ids, n in chunks:
+        part = gather(pool, layer, [(page_ids, n)])
+        parts.append(rope_rebase_bits(part, at, base))
+        at += n
+    if not parts:
+        return pool[layer, :0, :, 0, :]
+    return np.concatenate(parts, axis=0)
+
+
+# --------------------------------------------------------------------------
 # step 3 + 4: masked softmax attention and Impact for one request
 # --------------------------------------------------------------------------
 
@@ -217,8 +267,9 @@ def build_layer_pool(lay, inputs, bits_dtype):
 
 
 def run_workload_layer(lay, inputs, want_impact: bool, scale: float = None,
-                       keep_pool: bool = False) -> OracleResult:
-    """Oracle for one layer of a generated batch (all requests)."""
+                       keep_pool: bool = False, rope_base: float = None) -> OracleResult:
+    """Oracle for one layer of a generated batch (all requests). rope_base:
+    re-base the cached keys to their concatenated positions (None: as stored)."""
     w = lay.workload
     d = w.head_dim
     scale = 1.0 / np.sqrt(d) if scale is None else scale
@@ -236,7 +287,12 @@ def run_workload_layer(lay, inputs, want_impact: bool, scale: float = None,
     for b, cs in enumerate(lay.req_chunks):
         ql = lay.q_lens[b]
         chunks = [(lay.chunk_pages[c].numpy(), lay.chunk_len[c]) for c in cs]
-        kd = bits_to_f64(gather(pk, 0, chunks))
+        if rope_base is None:
+            kd = bits_to_f64(gather(pk, 0, chunks))
+        else:
+            if bits_dtype != np.uint16:
+                raise TypeError("re-basing is defined for bf16 caches")
+            kd = bits_to_f64(gather_rebased(pk, 0, chunks, rope_base))
         vd = bits_to_f64(gather(pv, 0, chunks))
         n_doc = kd.shape[0]
         kcat = np.concatenate([kd, kq_all[q0:q0 + ql]], axis=0)
