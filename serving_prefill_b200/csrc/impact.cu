@@ -16,7 +16,8 @@
 //   8 epilogue warps: two per TMEM lane quarter, each over half of the rows;
 //                   per key 2^(s c + b_row), with the row's normaliser folded
 //                   into the bias b_row = log2(1 / (l H_q)) - m2, summed on
-//                   MUFU exp2, the halves added in shared memory, atomicAdd
+//                   MUFU exp2 with packed fp32 pair arithmetic; each half
+//                   adds its column sum with one atomicAdd per key
 // The producer and MMA warps start while the kernels before this one finish
 // (programmatic dependent launch); the epilogue waits for their row
 // statistics.
@@ -36,8 +37,7 @@ constexpr int kITileBytes = kBN * kHeadDim * 2;     // K tile
 constexpr int kIHalf = kITileBytes / 2;
 constexpr int kIQHalf = kImpactRows * 128;          // 256 rows x 64 d (bf16) per d-half
 constexpr int kIQBytes = 2 * kIQHalf;
-constexpr int kImpThreads = 320;              // 8 epilogue + producer + MMA warps
-constexpr int kImpPolyPairsOf8 = 0;          // of every 8 column pairs, this many use the FMA-pipe exp2 (fastest: 0)
+constexpr int kImpThreads = 352;              // 8 epilogue + producer + MMA + RoPE warps
 
 struct ImpDesc {
   int32_t kind;      // 0 doc tile, 1 query-key tile
@@ -49,14 +49,14 @@ struct ImpDesc {
 
 struct ImpCtrl {
   uint64_t q_full, q_empty;
-  uint64_t kfull[kIKStages], kempty[kIKStages];
+  uint64_t kfull[kIKStages], kempty[kIKStages], kconv[kIKStages];
+  int32_t kchunk[kIKStages][kPagesPerTile];   // chunk-list entry per page of a K stage (-1: none)
   uint64_t s_full[2], s_free[2];
   uint64_t teardown;
   uint64_t desc_full[kIDescSlots], desc_empty[kIDescSlots];
   ImpDesc desc[kIDescSlots];
   ChunkCache chunks;
   alignas(16) float neg_m2[kImpactRows];   // per row: log2(1 / (l * H_q)) - m (log2 units; -inf: no row)
-  float red[2][kBN];                      // second-half column sums, per S buffer
   uint32_t tmem_base;
   int32_t abort;
   int32_t total_items;
@@ -131,7 +131,11 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   if (tid == 0) {
     mbar_init(&ctl->q_full, 1);
     mbar_init(&ctl->q_empty, 1);
-    for (int s = 0; s < kIKStages; ++s) { mbar_init(&ctl->kfull[s], 1); mbar_init(&ctl->kempty[s], 1); }
+    for (int s = 0; s < kIKStages; ++s) {
+      mbar_init(&ctl->kfull[s], 1);
+      mbar_init(&ctl->kempty[s], 1);
+      mbar_init(&ctl->kconv[s], 1);
+    }
     for (int s = 0; s < 2; ++s) { mbar_init(&ctl->s_full[s], 1); mbar_init(&ctl->s_free[s], 256); }
     mbar_init(&ctl->teardown, 1);
     for (int s = 0; s < kIDescSlots; ++s) { mbar_init(&ctl->desc_full[s], 1); mbar_init(&ctl->desc_empty[s], 8); }
@@ -231,25 +235,44 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (!mbar_wait(&ctl->s_full[buf], (t >> 1) & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
         const uint32_t col = tmem + lane_off + (buf ? 256u : 0u) + c0;
-        // 32-column chunks with the next chunk's TMEM load in flight while
-        // the current one is reduced
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        auto chunk = [&](const uint32_t (&u)[32], int cbase) {
+        // 32-column chunks with the next chunk's TMEM load in flight while the
+        // current one is reduced; per score one packed FMA (scale and the
+        // row's bias) per pair, one exp2 on MUFU, one packed add per pair
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
+        // doc tiles: every row sees every key, no mask
+        auto chunk_doc = [&](const uint32_t (&u)[32], int cbase) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float4 b = *reinterpret_cast<const float4*>(&ctl->neg_m2[c0 + cbase + j]);
+            const float2 e0 = ffma2(make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1])), sc2,
+                                    make_float2(b.x, b.y));
+            const float2 e1 = ffma2(make_float2(__uint_as_float(u[j + 2]), __uint_as_float(u[j + 3])), sc2,
+                                    make_float2(b.z, b.w));
+            const int a = (j >> 1) & 2;
+            acc[a] = fadd2(acc[a], make_float2(ex2(e0.x), ex2(e0.y)));
+            acc[a + 1] = fadd2(acc[a + 1], make_float2(ex2(e1.x), ex2(e1.y)));
+          }
+        };
+        // query-key tiles: row r sees this key from r >= rlim on (causal)
+        auto chunk_query = [&](const uint32_t (&u)[32], int cbase) {
 #pragma unroll
           for (int j = 0; j < 32; j += 4) {
             const int r0 = c0 + cbase + j;
-            const float4 bias = *reinterpret_cast<const float4*>(&ctl->neg_m2[r0]);
-            float e[4];
-            e[0] = fmaf(__uint_as_float(u[j]), p.scale_log2, bias.x);
-            e[1] = fmaf(__uint_as_float(u[j + 1]), p.scale_log2, bias.y);
-            e[2] = fmaf(__uint_as_float(u[j + 2]), p.scale_log2, bias.z);
-            e[3] = fmaf(__uint_as_float(u[j + 3]), p.scale_log2, bias.w);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float v = ((((j + q) >> 1) & 7) < kImpPolyPairsOf8) ? exp2_poly(e[q]) : ex2(e[q]);
-              if (kind != 0 && r0 + q < rlim) v = 0.f;
-              acc[q] += v;
-            }
+            const float4 b = *reinterpret_cast<const float4*>(&ctl->neg_m2[r0]);
+            const float2 e0 = ffma2(make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1])), sc2,
+                                    make_float2(b.x, b.y));
+            const float2 e1 = ffma2(make_float2(__uint_as_float(u[j + 2]), __uint_as_float(u[j + 3])), sc2,
+                                    make_float2(b.z, b.w));
+            float v0 = ex2(e0.x), v1 = ex2(e0.y), v2 = ex2(e1.x), v3 = ex2(e1.y);
+            if (r0 < rlim) v0 = 0.f;
+            if (r0 + 1 < rlim) v1 = 0.f;
+            if (r0 + 2 < rlim) v2 = 0.f;
+            if (r0 + 3 < rlim) v3 = 0.f;
+            const int a = (j >> 1) & 2;
+            acc[a] = fadd2(acc[a], make_float2(v0, v1));
+            acc[a + 1] = fadd2(acc[a + 1], make_float2(v2, v3));
           }
         };
         uint32_t ua[32], ub[32];
@@ -258,23 +281,20 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int c = 0; c < cols; c += 64) {
           const bool more_b = c + 32 < cols;
           if (more_b) tmem_ld32(col + c + 32, ub);
-          chunk(ua, c);
+          if (kind == 0) chunk_doc(ua, c); else chunk_query(ua, c);
           tmem_wait_ld();
           if (!more_b) break;
           const bool more_a = c + 64 < cols;
           if (more_a) tmem_ld32(col + c + 64, ua);
-          chunk(ub, c + 32);
+          if (kind == 0) chunk_doc(ub, c + 32); else chunk_query(ub, c + 32);
           tmem_wait_ld();
         }
         tc_fence_before();
         mbar_arrive(&ctl->s_free[buf]);
-        float total = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        if (half == 1) ctl->red[buf][k] = total;
-        named_bar_sync(2, 256);
-        if (half == 0) {
-          total += ctl->red[buf][k];
-          if (valid) atomicAdd(seg + lpos, total);
-        }
+        // each half adds its own column sum: no barrier between the halves
+        const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+        const float total = (a01.x + a01.y) + (a23.x + a23.y);
+        if (valid) atomicAdd(seg + lpos, total);
       }
       t_glob += n;
     }
@@ -335,6 +355,8 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           bad = 1;
           break;
         }
+        if (lane < kPagesPerTile) ctl->kchunk[s][lane] = (doc && pg.page >= 0) ? pg.chunk : -1;
+        __syncwarp();
         if (lane == 0) mbar_arrive_expect_tx(&ctl->kfull[s], kITileBytes);
         __syncwarp();
         uint8_t* dst = sK + s * kITileBytes;
@@ -361,8 +383,30 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (q_iter > 0) mbar_wait(&ctl->q_full, (q_iter - 1) & 1, &zero);
     }
     __syncwarp();
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ RoPE re-basing of the K tiles
+    if (p.rope) {
+      uint32_t t_glob = 0;
+      int bad = 0;
+      for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
+        const ImpItem it = decode_imp_item(p, prefix, w);
+        const int n = it.t_end - it.t_begin;
+        for (int i = 0; i < n; ++i) {
+          const uint32_t t = t_glob + i;
+          const int s = t % kIKStages;
+          if (!mbar_wait(&ctl->kfull[s], (t / kIKStages) & 1, abort_flag)) { bad = 1; break; }
+          rope_rotate_tile(sK + s * kITileBytes, ctl->kchunk[s], p.rope, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->kconv[s]);
+        }
+        t_glob += n;
+      }
+      if (bad && lane == 0) imp_abort(ctl, p.err);
+      __syncwarp();
+    }
   } else {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ MMA issuer (warp 9)
     if (lane == 0) {
       const uint32_t q_base = smem_u32(sQ);
       uint32_t t_glob = 0, q_iter = 0;
@@ -377,7 +421,10 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int i = 0; i < n; ++i) {
           const uint32_t t = t_glob + i;
           const int s = t % kIKStages;
-          if (!mbar_wait(&ctl->kfull[s], (t / kIKStages) & 1, abort_flag)) { bad = 1; break; }
+          if (!mbar_wait(p.rope ? &ctl->kconv[s] : &ctl->kfull[s], (t / kIKStages) & 1, abort_flag)) {
+            bad = 1;
+            break;
+          }
           if (t >= 2 && !mbar_wait(&ctl->s_free[t & 1], ((t - 2) >> 1) & 1, abort_flag)) { bad = 1; break; }
           tc_fence_after();
           const uint32_t k_base = smem_u32(sK + s * kITileBytes);
