@@ -68,9 +68,11 @@ typedef enum {
   RAG_ERR_TIMEOUT = 6,     /* device: a pipeline wait gave up                 */
   RAG_ERR_WORKSPACE = 7,   /* workspace missing or smaller than required      */
   RAG_ERR_GEOMETRY = 8,    /* device: chunk pages do not match its length     */
-  RAG_ERR_RANGE = 9        /* device: a bf16 V value of magnitude >= 65536
+  RAG_ERR_RANGE = 9,       /* device: a bf16 V value of magnitude >= 65536
                               (or inf/nan) met the fp16 PV product and was
                               saturated to +-65504; O is then inexact        */
+  RAG_ERR_NO_FREE_PAGES = 10 /* device: the copy-on-write recompute needs more
+                              private pages than the free list holds          */
 } rag_status;
 
 typedef enum { RAG_BF16 = 0, RAG_F32 = 1 } rag_dtype;
@@ -178,6 +180,26 @@ RAG_API rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer
                                   float* row_lse, float* impact, void* workspace, size_t workspace_bytes,
                                   void* stream);
 
+/* rag_fused_prefill_attn with the cached keys re-based to their positions in
+ * the concatenated sequence (TurboRAG page, "Implementation": with rotary
+ * position embeddings, the position ids of the offline precompute and of
+ * inference must agree). Each chunk's cached K is taken to carry RoPE at its
+ * chunk-local positions 0 .. n_c - 1; chunk-list entry e of a request starts at
+ * offset o_e (the doc tokens of the request's entries before it), and every
+ * key of it is turned by o_e positions: rotary pair i (channels i and i + 64)
+ * by the angle o_e * rope_base^(-2i/128). The rotated key is rounded once to
+ * bf16 (the cache dtype) before the products. The query block's q, kq are
+ * expected with RoPE at their positions N_doc,b + j already applied. The pool
+ * itself is not modified (the rotation happens on the way from HBM to the
+ * tensor core, in attention and in the Impact pass alike). rope_base > 1
+ * (10000 for Llama-2, 500000 for Llama-3); bf16 pools only. The workspace
+ * holds a (cos, sin) table per chunk-list entry, rebuilt by every call. */
+RAG_API rag_status rag_fused_prefill_attn_rope(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch,
+                                               const void* q, int32_t num_q_heads, const void* kq, const void* vq,
+                                               float sm_scale, double rope_base, void* o, float* row_lse,
+                                               float* impact, void* workspace, size_t workspace_bytes,
+                                               void* stream);
+
 /* Same computation as rag_fused_prefill_attn, for callers that cannot
  * allocate device memory (a runtime that gives a plugin only its input and
  * output buffers, a deployment whose device memory is planned once at start-up,
@@ -228,6 +250,70 @@ RAG_API int32_t rag_recompute_count(int32_t n_doc, double r);
 RAG_API rag_status rag_impact_topk(const float* impact, const rag_batch* batch, double r, int32_t k_cap,
                            int32_t* topk_idx, float* topk_val, int32_t* k_out, void* stream);
 
+/* ---- Selective recompute of the chosen tokens' K and V ---------------------
+ * CacheBlend page, "Contributions" (only the tokens of high attention impact
+ * are recomputed when the cached KV are fused) and "How it works" (after the
+ * high-Impact tokens are found, their KV values are recomputed and generation
+ * runs on the fused cache). A chunk's pages are shared by every request that
+ * retrieved it, so the recompute never writes them: each page reference that
+ * holds a selected token gets a private page (copy on write) and the
+ * request's page table is rewritten to point at it.
+ *
+ * Use: rag_impact_topk -> rag_recompute_plan (once) -> rag_recompute_kv for
+ * every layer, with the layer's hidden states of the selected tokens and its
+ * K/V projection weights -> attention with page_ids_out as the page table. */
+
+/* Bytes of the plan buffer for this batch and top-k row length (0 on invalid
+ * arguments). */
+RAG_API size_t rag_recompute_plan_size(const rag_batch* batch, int32_t k_cap);
+
+/* Plan the copy-on-write pages and the destination of every selected token.
+ * topk_idx [B][k_cap], k [B]: as written by rag_impact_topk (device int32);
+ *   request b's selected doc positions are topk_idx[b][0 .. k[b]-1].
+ * free_pages [n_free] device int32: page ids of the pool the caller reserved
+ *   for private copies (distinct, unused by any page table). They are handed
+ *   out in ascending order of page reference over the whole batch.
+ * x_by_selection: 0 -> the hidden state of request b's position i is row
+ *   chunk_doc_off[req_chunk_off[b]] + i of the x array given to
+ *   rag_recompute_kv ([total_doc][d_model], every doc token of the batch);
+ *   1 -> row t, the token's rank in the batch's selection (requests in order,
+ *   then topk order: [sum_b k[b]][d_model]).
+ * page_ids_out [num_page_refs] device int32: the batch's page table after copy
+ *   on write (may be batch->page_ids itself, updated in place).
+ * plan: device buffer of rag_recompute_plan_size bytes, 256-byte aligned,
+ *   written here and read by rag_recompute_kv; one plan serves every layer.
+ * If the selection needs more private pages than n_free, nothing is remapped
+ * (page_ids_out = page_ids), rag_recompute_kv then writes nothing, and
+ * rag_recompute_status reports RAG_ERR_NO_FREE_PAGES with the count needed.
+ * A selected position outside its request is skipped (RAG_ERR_GEOMETRY). */
+RAG_API rag_status rag_recompute_plan(const rag_batch* batch, const int32_t* topk_idx, int32_t k_cap,
+                                      const int32_t* k, const int32_t* free_pages, int32_t n_free,
+                                      int32_t x_by_selection, int32_t* page_ids_out, void* plan,
+                                      size_t plan_bytes, void* stream);
+
+/* One layer of the recompute (bf16 pool, head_dim 128):
+ *   every private page first receives, for this layer, the K and V of every
+ *   slot that is not selected from the page it replaces (all KV heads);
+ *   every selected token's rows are recomputed from its hidden state:
+ *   K = x W_K^T, V = x W_V^T (fp32 accumulation, one rounding to bf16), split
+ *   into num_kv_heads heads of 128, and stored into its slot of its private
+ *   page. The copy and the recompute never write the same bytes.
+ * x   [x_rows][d_model] bf16 device, rows as x_by_selection of the plan says;
+ * w_k, w_v [num_kv_heads * 128][d_model] bf16 device (a linear layer's weight);
+ * d_model a multiple of 64. batch and k_cap as given to rag_recompute_plan.
+ * Device problems (a free page id outside the pool, a row past x_rows, a wait
+ * that gave up) are recorded in the plan and reported by rag_recompute_status. */
+RAG_API rag_status rag_recompute_kv(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch, int32_t k_cap,
+                                    const void* plan, size_t plan_bytes, const void* x, int64_t x_rows,
+                                    int32_t d_model, const void* w_k, const void* w_v, void* stream);
+
+/* Synchronise `stream` and read the plan's counts: counts[0] selected tokens
+ * recomputed, counts[1] private pages used, counts[2] private pages the
+ * selection needs (optional, 3 int32, host). Returns RAG_OK or the most
+ * severe of RAG_ERR_TIMEOUT, RAG_ERR_NO_FREE_PAGES, RAG_ERR_PAGE_OOB,
+ * RAG_ERR_GEOMETRY. */
+RAG_API rag_status rag_recompute_status(const void* plan, int32_t* counts, void* stream);
+
 /* Synchronise `stream`, read and clear the workspace error word. Returns
  * RAG_OK when the device reported nothing, else the most severe of
  * RAG_ERR_TIMEOUT, RAG_ERR_PAGE_OOB, RAG_ERR_GEOMETRY, RAG_ERR_RANGE; *bits
@@ -252,7 +338,9 @@ RAG_API int64_t rag_launch_count(void);
 /* Per-kernel timing: when enabled, every launch is bracketed by CUDA events
  * on its stream. rag_profile_collect synchronises, writes the summed device
  * milliseconds and launch counts per kernel kind (0 pool write, 1 attention,
- * 2 split combine, 3 impact, 4 top-k, 5 fp32 attention, 6 fp32 impact) into
+ * 2 split combine, 3 impact, 4 top-k, 5 fp32 attention, 6 fp32 impact,
+ * 7 recompute plan, 8 recompute page copy, 9 recompute projection,
+ * 10 RoPE table) into
  * the first n_kinds entries of ms and launches (either may be NULL), and
  * resets the record. */
 RAG_API void rag_profile_enable(int32_t on);

@@ -14,6 +14,7 @@ from .rag import (  # noqa: F401
     new_workspace,
     rag_abi_version,
     rag_fused_prefill_attn,
+    rag_fused_prefill_attn_rope,
     rag_impact_topk,
     rag_kv_pool_write,
     rag_last_device_error,
@@ -23,6 +24,10 @@ from .rag import (  # noqa: F401
     rag_profile_peek,
     rag_profile_enable,
     rag_recompute_count,
+    rag_recompute_kv,
+    rag_recompute_plan,
+    rag_recompute_plan_size,
+    rag_recompute_status,
     rag_workspace_size,
     topk_capacity,
 )

@@ -79,6 +79,7 @@ struct FwdParams {
   float* impact_zero;
   int64_t impact_len;
   int64_t max_items;              // partial slots the workspace holds
+  const float2* rope;             // per chunk-list entry, 64 (cos, sin) pairs; null: keys used as stored
 };
 struct CombineParams {
   BatchDev batch;
@@ -100,6 +101,7 @@ struct ImpactParams {
   const float* row_il;
   float* impact;
   int32_t* err;
+  const float2* rope;             // as FwdParams::rope
 };
 struct TopkParams {
   BatchDev batch;
@@ -138,9 +140,73 @@ struct PoolWriteParams {
   int32_t row_bytes;
 };
 
+// Selective recompute. The plan buffer (int32 words, each region 64-word
+// aligned) that the plan kernel writes and the copy and GEMM kernels read:
+//   header   16 words: n_tok, n_cow, n_needed, error bits
+//   x_row    [max_tok]  hidden-state row of selected token t (-1: skipped)
+//   dst      [max_tok]  private page * 16 + slot of token t (slot only, before the pages are known)
+//   ref      [max_tok]  page reference of token t (-1: skipped)
+//   cow_src  [max_cow]  page copied from
+//   cow_dst  [max_cow]  private page copied to
+//   cow_mask [max_cow]  selected slots of that page (bit s: slot s), which the copy leaves alone
+//   flags    [page_refs] selected-slot mask per page reference
+// max_tok = B * k_cap, max_cow = page_refs.
+struct RcPlanLayout {
+  int64_t x_row, dst, ref, cow_src, cow_dst, cow_mask, flags, words;
+};
+__host__ __device__ inline int64_t align64w(int64_t x) { return (x + 63) & ~int64_t(63); }
+__host__ __device__ inline RcPlanLayout rc_plan_layout(int64_t max_tok, int64_t page_refs) {
+  RcPlanLayout l;
+  int64_t at = 64;
+  l.x_row = at; at = align64w(at + max_tok);
+  l.dst = at; at = align64w(at + max_tok);
+  l.ref = at; at = align64w(at + max_tok);
+  l.cow_src = at; at = align64w(at + page_refs);
+  l.cow_dst = at; at = align64w(at + page_refs);
+  l.cow_mask = at; at = align64w(at + page_refs);
+  l.flags = at; at = align64w(at + page_refs);
+  l.words = at;
+  return l;
+}
+enum : int32_t { kRcHdrTok = 0, kRcHdrCow = 1, kRcHdrNeeded = 2, kRcHdrErr = 3 };
+enum : int32_t { kRcErrNoFree = 16 };   // error bit beyond the device error bits: too few free pages
+
+struct RcPlanParams {
+  BatchDev batch;
+  const int32_t* topk_idx;
+  const int32_t* k;
+  const int32_t* free_pages;
+  int32_t* page_ids_out;
+  int32_t* plan;
+  RcPlanLayout lay;
+  int32_t k_cap, n_free, by_selection;
+};
+struct RcCopyParams {
+  uint8_t* pool_k;
+  uint8_t* pool_v;
+  int32_t* plan;
+  RcPlanLayout lay;
+  int32_t layer, num_pages, num_kv_heads;
+};
+struct RcGemmParams {
+  __nv_bfloat16* pool_k;
+  __nv_bfloat16* pool_v;
+  int32_t* plan;
+  RcPlanLayout lay;
+  int32_t layer, num_pages, num_kv_heads, d_model;
+  int32_t x_rows;
+  int64_t max_tok;
+};
+
+cudaError_t launch_rc_plan(const RcPlanParams&, cudaStream_t);
+cudaError_t launch_rc_copy(const RcCopyParams&, int grid, cudaStream_t);
+cudaError_t launch_rc_gemm(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const RcGemmParams&, int grid,
+                           cudaStream_t);
+
 cudaError_t launch_attn_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                             const CUtensorMap&, const FwdParams&, int, cudaStream_t);
 cudaError_t launch_attn_combine(const CombineParams&, int, int, cudaStream_t);
+cudaError_t launch_rope_table(const BatchDev&, double base, float2* table, cudaStream_t);
 cudaError_t launch_impact(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const ImpactParams&, int,
                           cudaStream_t);
 cudaError_t launch_topk(const TopkParams&, int, int, cudaStream_t);

@@ -19,11 +19,12 @@ namespace rag {
 
 constexpr int kSimtMaxKeysHost = 8192;
 constexpr int kTopkMaxKHost = 16384;
+constexpr int kRcMinDModel = 64;
 
 // ------------------------------------------------------------ profiling
 
 enum Kind { kKindPoolWrite = 0, kKindAttn, kKindCombine, kKindImpact, kKindTopk, kKindSimtAttn, kKindSimtImpact,
-            kNumKinds };
+            kKindRcPlan, kKindRcCopy, kKindRcGemm, kKindRope, kNumKinds };
 
 struct ProfRecord {
   int kind;
@@ -220,7 +221,8 @@ static BatchDev to_dev(const rag_batch& b) {
 static size_t workspace_bytes_for(const rag_kv_pool& pool, const rag_batch& b, int num_q_heads) {
   const int G = num_q_heads / pool.num_kv_heads;
   const Plan pf = plan_split(b, pool.num_kv_heads, G, kFwdRows, num_sms());
-  return ws_layout(b.total_q, num_q_heads, pool.dtype == RAG_BF16 ? pf.max_items : 0).total;
+  const bool bf16 = pool.dtype == RAG_BF16;
+  return ws_layout(b.total_q, num_q_heads, bf16 ? pf.max_items : 0, bf16 ? b.num_chunks : 0).total;
 }
 
 }  // namespace rag
@@ -243,6 +245,7 @@ const char* rag_status_string(int32_t s) {
     case RAG_ERR_WORKSPACE: return "workspace missing or too small";
     case RAG_ERR_GEOMETRY: return "chunk page count does not match its length";
     case RAG_ERR_RANGE: return "a V value beyond the fp16 range was saturated";
+    case RAG_ERR_NO_FREE_PAGES: return "too few free pages for the copy-on-write recompute";
     default: return "unknown status";
   }
 }
@@ -294,10 +297,16 @@ rag_status rag_workspace_init(void* workspace, size_t workspace_bytes, void* str
                                                                                             : RAG_ERR_CUDA;
 }
 
-rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch, const void* q,
-                                  int32_t num_q_heads, const void* kq, const void* vq, float sm_scale, void* o,
-                                  float* row_lse, float* impact, void* workspace, size_t workspace_bytes,
-                                  void* stream) {
+}  // extern "C"
+
+namespace rag {
+
+// The fused prefill of one layer; rope_base > 0 re-bases the cached keys to
+// their concatenated positions (bf16 pools only).
+static rag_status fused_prefill(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch, const void* q,
+                                int32_t num_q_heads, const void* kq, const void* vq, float sm_scale,
+                                double rope_base, void* o, float* row_lse, float* impact, void* workspace,
+                                size_t workspace_bytes, void* stream) {
   rag_status st = check_pool(pool);
   if (st != RAG_OK) return st;
   st = check_batch(batch);
@@ -327,8 +336,9 @@ rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const 
   }
 
   if (pool->dtype == RAG_F32) {
+    if (rope_base > 0.0) return RAG_ERR_UNSUPPORTED;
     if (b.max_doc + b.max_q > kSimtMaxKeysHost) return RAG_ERR_UNSUPPORTED;
-    const WsLayout wl = ws_layout(b.total_q, num_q_heads, 0);
+    const WsLayout wl = ws_layout(b.total_q, num_q_heads, 0, 0);
     SimtParams p;
     p.batch = to_dev(b);
     p.num_pages = pool->num_pages;
@@ -368,7 +378,7 @@ rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const 
   if (kBM % G != 0) return RAG_ERR_UNSUPPORTED;
   const int sms = num_sms();
   const Plan pf = plan_split(b, pool->num_kv_heads, G, kFwdRows, sms);
-  const WsLayout wl = ws_layout(b.total_q, num_q_heads, pf.max_items);
+  const WsLayout wl = ws_layout(b.total_q, num_q_heads, pf.max_items, b.num_chunks);
   const int H_kv = pool->num_kv_heads;
   const uint64_t pool_rows = uint64_t(pool->num_layers) * pool->num_pages * H_kv * kPage;
 
@@ -393,6 +403,14 @@ rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const 
   int32_t* item_prefix = reinterpret_cast<int32_t*>(ws + wl.off_prefix);
   float* part = reinterpret_cast<float*>(ws + wl.off_part);
   const float scale_log2 = scale * 1.4426950408889634f;
+  float2* rope = nullptr;
+  if (rope_base > 0.0) {
+    rope = reinterpret_cast<float2*>(ws + wl.off_rope);
+    LaunchScope ls(kKindRope, s);
+    cudaError_t e = launch_rope_table(to_dev(b), rope_base, rope, s);
+    ls.done(e);
+    if (e != cudaSuccess) return RAG_ERR_CUDA;
+  }
 
   FwdParams fp;
   fp.batch = to_dev(b);
@@ -414,6 +432,7 @@ rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const 
   fp.impact_zero = impact;
   fp.impact_len = impact ? impact_len : 0;
   fp.max_items = pf.max_items;
+  fp.rope = rope;
   {
     LaunchScope ls(kKindAttn, s);
     cudaError_t e = launch_attn_fwd(tm_q, tm_k, tm_v, tm_kq, tm_vq, fp, pf.grid, s);
@@ -454,12 +473,34 @@ rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const 
     ip.row_il = row_il;
     ip.impact = impact;
     ip.err = err;
+    ip.rope = rope;
     LaunchScope ls(kKindImpact, s);
     cudaError_t e = launch_impact(tm_q, tm_k, tm_kq, ip, pi.grid, s);
     ls.done(e);
     if (e != cudaSuccess) return RAG_ERR_CUDA;
   }
   return RAG_OK;
+}
+
+}  // namespace rag
+
+extern "C" {
+
+rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch, const void* q,
+                                  int32_t num_q_heads, const void* kq, const void* vq, float sm_scale, void* o,
+                                  float* row_lse, float* impact, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  return fused_prefill(pool, layer, batch, q, num_q_heads, kq, vq, sm_scale, 0.0, o, row_lse, impact, workspace,
+                       workspace_bytes, stream);
+}
+
+rag_status rag_fused_prefill_attn_rope(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch,
+                                       const void* q, int32_t num_q_heads, const void* kq, const void* vq,
+                                       float sm_scale, double rope_base, void* o, float* row_lse, float* impact,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (!(rope_base > 1.0) || !std::isfinite(rope_base)) return RAG_ERR_INVALID_ARG;
+  return fused_prefill(pool, layer, batch, q, num_q_heads, kq, vq, sm_scale, rope_base, o, row_lse, impact,
+                       workspace, workspace_bytes, stream);
 }
 
 rag_status rag_impact_topk(const float* impact, const rag_batch* batch, double r, int32_t k_cap, int32_t* topk_idx,
@@ -487,6 +528,130 @@ rag_status rag_impact_topk(const float* impact, const rag_batch* batch, double r
   cudaError_t e = launch_topk(p, b.num_requests, p.k_max, s);
   ls.done(e);
   return e == cudaSuccess ? RAG_OK : RAG_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ selective recompute
+
+size_t rag_recompute_plan_size(const rag_batch* batch, int32_t k_cap) {
+  if (check_batch(batch) != RAG_OK || k_cap < 1) return 0;
+  const RcPlanLayout l = rc_plan_layout(int64_t(batch->num_requests) * k_cap, batch->num_page_refs);
+  return size_t(l.words) * sizeof(int32_t);
+}
+
+rag_status rag_recompute_plan(const rag_batch* batch, const int32_t* topk_idx, int32_t k_cap, const int32_t* k,
+                              const int32_t* free_pages, int32_t n_free, int32_t x_by_selection,
+                              int32_t* page_ids_out, void* plan, size_t plan_bytes, void* stream) {
+  rag_status st = check_batch(batch);
+  if (st != RAG_OK) return st;
+  if (k_cap < 1 || n_free < 0) return RAG_ERR_SHAPE;
+  const rag_batch& b = *batch;
+  if (!plan || (reinterpret_cast<uintptr_t>(plan) & 255u)) return RAG_ERR_WORKSPACE;
+  if (plan_bytes < rag_recompute_plan_size(batch, k_cap)) return RAG_ERR_WORKSPACE;
+  if (b.num_requests > 0 && (!topk_idx || !k)) return RAG_ERR_INVALID_ARG;
+  if (b.num_page_refs > 0 && !page_ids_out) return RAG_ERR_INVALID_ARG;
+  if (n_free > 0 && !free_pages) return RAG_ERR_INVALID_ARG;
+  RcPlanParams p;
+  p.batch = to_dev(b);
+  p.topk_idx = topk_idx;
+  p.k = k;
+  p.free_pages = free_pages;
+  p.page_ids_out = page_ids_out;
+  p.plan = static_cast<int32_t*>(plan);
+  p.lay = rc_plan_layout(int64_t(b.num_requests) * k_cap, b.num_page_refs);
+  p.k_cap = k_cap;
+  p.n_free = n_free;
+  p.by_selection = x_by_selection ? 1 : 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  LaunchScope ls(kKindRcPlan, s);
+  cudaError_t e = launch_rc_plan(p, s);
+  ls.done(e);
+  return e == cudaSuccess ? RAG_OK : RAG_ERR_CUDA;
+}
+
+rag_status rag_recompute_kv(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch, int32_t k_cap,
+                            const void* plan, size_t plan_bytes, const void* x, int64_t x_rows, int32_t d_model,
+                            const void* w_k, const void* w_v, void* stream) {
+  rag_status st = check_pool(pool);
+  if (st != RAG_OK) return st;
+  st = check_batch(batch);
+  if (st != RAG_OK) return st;
+  if (pool->dtype != RAG_BF16) return RAG_ERR_UNSUPPORTED;
+  if (layer < 0 || layer >= pool->num_layers) return RAG_ERR_INVALID_ARG;
+  if (k_cap < 1) return RAG_ERR_SHAPE;
+  if (d_model < kRcMinDModel || d_model % 64 != 0 || d_model > (1 << 20)) return RAG_ERR_UNSUPPORTED;
+  if (x_rows < 1 || x_rows >= (int64_t(1) << 31)) return RAG_ERR_SHAPE;
+  if (!plan || (reinterpret_cast<uintptr_t>(plan) & 255u)) return RAG_ERR_WORKSPACE;
+  if (plan_bytes < rag_recompute_plan_size(batch, k_cap)) return RAG_ERR_WORKSPACE;
+  if (!x || !w_k || !w_v || !aligned16(x) || !aligned16(w_k) || !aligned16(w_v)) return RAG_ERR_INVALID_ARG;
+  const rag_batch& b = *batch;
+  const int H_kv = pool->num_kv_heads;
+  const RcPlanLayout lay = rc_plan_layout(int64_t(b.num_requests) * k_cap, b.num_page_refs);
+  const int64_t max_tok = int64_t(b.num_requests) * k_cap;
+  if (max_tok == 0) return RAG_OK;
+  CUtensorMap tm_x, tm_wk, tm_wv;
+  {
+    const uint64_t dx[2] = {uint64_t(d_model), uint64_t(x_rows)};
+    const uint64_t sx[1] = {uint64_t(d_model) * 2};
+    const uint32_t bx[2] = {64u, 1u};
+    const uint64_t dw[2] = {uint64_t(d_model), uint64_t(H_kv) * kHeadDim};
+    const uint32_t bw[2] = {64u, 128u};
+    if (!make_map(&tm_x, x, 2, dx, sx, bx) || !make_map(&tm_wk, w_k, 2, dw, sx, bw) ||
+        !make_map(&tm_wv, w_v, 2, dw, sx, bw))
+      return RAG_ERR_CUDA;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = num_sms();
+  {
+    RcCopyParams cp;
+    cp.pool_k = static_cast<uint8_t*>(pool->k);
+    cp.pool_v = static_cast<uint8_t*>(pool->v);
+    cp.plan = static_cast<int32_t*>(const_cast<void*>(plan));
+    cp.lay = lay;
+    cp.layer = layer;
+    cp.num_pages = pool->num_pages;
+    cp.num_kv_heads = H_kv;
+    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(int64_t(4) * sms, b.num_page_refs)));
+    LaunchScope ls(kKindRcCopy, s);
+    cudaError_t e = launch_rc_copy(cp, grid, s);
+    ls.done(e);
+    if (e != cudaSuccess) return RAG_ERR_CUDA;
+  }
+  RcGemmParams gp;
+  gp.pool_k = static_cast<__nv_bfloat16*>(pool->k);
+  gp.pool_v = static_cast<__nv_bfloat16*>(pool->v);
+  gp.plan = static_cast<int32_t*>(const_cast<void*>(plan));
+  gp.lay = lay;
+  gp.layer = layer;
+  gp.num_pages = pool->num_pages;
+  gp.num_kv_heads = H_kv;
+  gp.d_model = d_model;
+  gp.x_rows = int32_t(x_rows);
+  gp.max_tok = max_tok;
+  const int64_t tiles_bound = ((max_tok + 127) / 128) * 2 * H_kv;
+  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(sms, tiles_bound)));
+  LaunchScope ls(kKindRcGemm, s);
+  cudaError_t e = launch_rc_gemm(tm_x, tm_wk, tm_wv, gp, grid, s);
+  ls.done(e);
+  return e == cudaSuccess ? RAG_OK : RAG_ERR_CUDA;
+}
+
+rag_status rag_recompute_status(const void* plan, int32_t* counts, void* stream) {
+  if (!plan) return RAG_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t hdr[4] = {0, 0, 0, 0};
+  if (cudaMemcpyAsync(hdr, plan, sizeof(hdr), cudaMemcpyDeviceToHost, s) != cudaSuccess) return RAG_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RAG_ERR_CUDA;
+  if (counts) {
+    counts[0] = hdr[kRcHdrTok];
+    counts[1] = hdr[kRcHdrCow];
+    counts[2] = hdr[kRcHdrNeeded];
+  }
+  const int32_t bits = hdr[kRcHdrErr];
+  if (bits & kDevErrTimeout) return RAG_ERR_TIMEOUT;
+  if (bits & kRcErrNoFree) return RAG_ERR_NO_FREE_PAGES;
+  if (bits & kDevErrPage) return RAG_ERR_PAGE_OOB;
+  if (bits & kDevErrGeometry) return RAG_ERR_GEOMETRY;
+  return RAG_OK;
 }
 
 rag_status rag_last_device_error(void* workspace, int32_t* bits, void* stream) {

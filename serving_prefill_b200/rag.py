@@ -18,13 +18,15 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librag.so")
 
 RAG_BF16, RAG_F32 = 0, 1
 PAGE_SIZE = 16
-KERNEL_KINDS = ("pool_write", "attn", "combine", "impact", "topk", "simt_attn", "simt_impact")
+KERNEL_KINDS = ("pool_write", "attn", "combine", "impact", "topk", "simt_attn", "simt_impact", "rc_plan", "rc_copy",
+                "rc_gemm", "rope_table")
 
 STATUS = {
     0: "ok", 1: "invalid argument", 2: "inconsistent shape", 3: "page id outside the pool",
     4: "unsupported configuration", 5: "CUDA runtime error", 6: "device pipeline wait timed out",
     7: "workspace missing or too small", 8: "chunk page count does not match its length",
     9: "a V value beyond the fp16 range was saturated",
+    10: "too few free pages for the copy-on-write recompute",
 }
 
 
@@ -59,6 +61,9 @@ EXPORTS = {
     "rag_fused_prefill_attn": (c_int32, [POINTER(RagKVPool), c_int32, POINTER(RagBatch), c_void_p, c_int32,
                                          c_void_p, c_void_p, c_float, c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_size_t, c_void_p]),
+    "rag_fused_prefill_attn_rope": (c_int32, [POINTER(RagKVPool), c_int32, POINTER(RagBatch), c_void_p, c_int32,
+                                              c_void_p, c_void_p, c_float, c_double, c_void_p, c_void_p, c_void_p,
+                                              c_void_p, c_size_t, c_void_p]),
     "rag_fused_prefill_attn_static": (c_int32, [POINTER(RagKVPool), c_int32, POINTER(RagBatch), c_void_p,
                                                 c_int32, c_void_p, c_void_p, c_float, c_void_p, c_void_p,
                                                 c_void_p, c_void_p, c_void_p]),
@@ -67,6 +72,12 @@ EXPORTS = {
                                   c_void_p]),
     "rag_last_device_error": (c_int32, [c_void_p, c_void_p, c_void_p]),
     "rag_selftest_wait_timeout": (c_int32, [c_void_p, c_int64, c_void_p]),
+    "rag_recompute_plan_size": (c_size_t, [POINTER(RagBatch), c_int32]),
+    "rag_recompute_plan": (c_int32, [POINTER(RagBatch), c_void_p, c_int32, c_void_p, c_void_p, c_int32, c_int32,
+                                     c_void_p, c_void_p, c_size_t, c_void_p]),
+    "rag_recompute_kv": (c_int32, [POINTER(RagKVPool), c_int32, POINTER(RagBatch), c_int32, c_void_p, c_size_t,
+                                   c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]),
+    "rag_recompute_status": (c_int32, [c_void_p, c_void_p, c_void_p]),
     "rag_launch_count": (c_int64, []),
     "rag_profile_enable": (None, [c_int32]),
     "rag_profile_collect": (c_int32, [c_void_p, c_void_p, c_int32]),
@@ -201,6 +212,17 @@ def rag_fused_prefill_attn(pool: KVPool, layer: int, batch: Batch, q: torch.Tens
            "rag_fused_prefill_attn")
 
 
+def rag_fused_prefill_attn_rope(pool: KVPool, layer: int, batch: Batch, q: torch.Tensor, kq: torch.Tensor,
+                                vq: torch.Tensor, o: torch.Tensor, workspace: torch.Tensor, rope_base: float,
+                                impact: torch.Tensor = None, row_lse: torch.Tensor = None, sm_scale: float = 0.0,
+                                stream=None):
+    num_q_heads = q.shape[1] if q.dim() == 3 else 0
+    _check(lib().rag_fused_prefill_attn_rope(ctypes.byref(pool.c), layer, ctypes.byref(batch.c), _ptr(q),
+                                             num_q_heads, _ptr(kq), _ptr(vq), sm_scale, rope_base, _ptr(o),
+                                             _ptr(row_lse), _ptr(impact), _ptr(workspace), workspace.numel(),
+                                             _stream(stream)), "rag_fused_prefill_attn_rope")
+
+
 def rag_fused_prefill_attn_static(pool: KVPool, layer: int, batch: Batch, q: torch.Tensor, kq: torch.Tensor,
                                   vq: torch.Tensor, o: torch.Tensor, impact: torch.Tensor = None,
                                   row_lse: torch.Tensor = None, device_err: torch.Tensor = None,
@@ -229,6 +251,33 @@ def rag_last_device_error(workspace: torch.Tensor, stream=None) -> tuple:
 def rag_selftest_wait_timeout(device_err: torch.Tensor, limit_ns: int, stream=None):
     _check(lib().rag_selftest_wait_timeout(_ptr(device_err), limit_ns, _stream(stream)),
            "rag_selftest_wait_timeout")
+
+
+def rag_recompute_plan_size(batch: Batch, k_cap: int) -> int:
+    n = lib().rag_recompute_plan_size(ctypes.byref(batch.c), k_cap)
+    if n == 0:
+        raise RagError(1, "rag_recompute_plan_size")
+    return n
+
+
+def rag_recompute_plan(batch: Batch, topk_idx: torch.Tensor, k_cap: int, k: torch.Tensor, free_pages: torch.Tensor,
+                       page_ids_out: torch.Tensor, plan: torch.Tensor, x_by_selection: bool = False, stream=None):
+    _check(lib().rag_recompute_plan(ctypes.byref(batch.c), _ptr(topk_idx), k_cap, _ptr(k), _ptr(free_pages),
+                                    free_pages.numel(), 1 if x_by_selection else 0, _ptr(page_ids_out), _ptr(plan),
+                                    plan.numel() * plan.element_size(), _stream(stream)), "rag_recompute_plan")
+
+
+def rag_recompute_kv(pool: KVPool, layer: int, batch: Batch, k_cap: int, plan: torch.Tensor, x: torch.Tensor,
+                     w_k: torch.Tensor, w_v: torch.Tensor, stream=None):
+    _check(lib().rag_recompute_kv(ctypes.byref(pool.c), layer, ctypes.byref(batch.c), k_cap, _ptr(plan),
+                                  plan.numel() * plan.element_size(), _ptr(x), x.shape[0], x.shape[1], _ptr(w_k),
+                                  _ptr(w_v), _stream(stream)), "rag_recompute_kv")
+
+
+def rag_recompute_status(plan: torch.Tensor, stream=None) -> tuple:
+    counts = (c_int32 * 3)()
+    st = lib().rag_recompute_status(_ptr(plan), ctypes.cast(counts, c_void_p), _stream(stream))
+    return st, (counts[0], counts[1], counts[2])
 
 
 def rag_launch_count() -> int:

@@ -22,12 +22,12 @@ TIE_RTOL = 1e-4
 class DeviceCase:
     """A workload's pool (the given layers), batch and engine on the GPU."""
 
-    def __init__(self, w, lay=None, layers=None, device="cuda"):
+    def __init__(self, w, lay=None, layers=None, device="cuda", spare_pages=0):
         self.w = w
         self.lay = make_layout(w) if lay is None else lay
         self.layers = list(range(w.num_layers)) if layers is None else list(layers)
-        self.pool = KVPool(w.num_layers, self.lay.num_pages, w.num_kv_heads, w.head_dim, dtype=w.torch_dtype,
-                           device=device)
+        self.pool = KVPool(w.num_layers, self.lay.num_pages + spare_pages, w.num_kv_heads, w.head_dim,
+                           dtype=w.torch_dtype, device=device)
         self.batch = Batch(self.lay.req_chunk_off, self.lay.chunk_doc_off, self.lay.chunk_page_off,
                            self.lay.page_ids, self.lay.q_off, device=device)
         self.engine = PrefillEngine(self.pool, self.batch, w.num_q_heads, w.r, dtype=w.torch_dtype, device=device)

@@ -14,6 +14,7 @@ from .rag import (  # noqa: F401
     LayerInputs,
     RecomputeInputs,
     make_recompute_inputs,
+    random_selection,
     make_layout,
     make_layer_inputs,
     get_workload,

@@ -311,10 +311,25 @@ class RecomputeInputs:
     w_v: torch.Tensor
 
 
-def make_recompute_inputs(w: Workload, lay: BatchLayout, layer: int) -> RecomputeInputs:
+def make_recompute_inputs(w: Workload, lay: BatchLayout, layer: int, rows: int = None) -> RecomputeInputs:
+    """rows: hidden-state rows to draw (default: one per doc token of the batch;
+    fewer when the caller indexes them by selection rank)."""
     n_out = w.num_kv_heads * w.head_dim
     std = 1.0 / float(w.d_model) ** 0.5
-    x = torch.randn(lay.total_doc, w.d_model, generator=_gen(w.seed, _T_X, layer)).to(torch.bfloat16)
+    n_rows = lay.total_doc if rows is None else rows
+    x = torch.randn(n_rows, w.d_model, generator=_gen(w.seed, _T_X, layer)).to(torch.bfloat16)
     wk = (torch.randn(n_out, w.d_model, generator=_gen(w.seed, _T_WK, layer)) * std).to(torch.bfloat16)
     wv = (torch.randn(n_out, w.d_model, generator=_gen(w.seed, _T_WV, layer)) * std).to(torch.bfloat16)
     return RecomputeInputs(x=x, w_k=wk, w_v=wv)
+
+
+def random_selection(doc_lens, counts, seed: int) -> list:
+    """Seeded stand-in for a top-k result: per request, counts[b] distinct doc
+    positions in random order (a selection lists positions by impact rank,
+    which is unrelated to position order)."""
+    g = _gen(seed, 123)
+    out = []
+    for n, k in zip(doc_lens, counts):
+        k = min(int(k), int(n))
+        out.append(torch.randperm(int(n), generator=g)[:k].tolist() if n > 0 else [])
+    return out
