@@ -406,6 +406,345 @@ def run_e2e(args, w, lay, layer_inputs, rep, device, world):
             "d2h_bytes_per_step": d2h, "steps": steps}
 
 
+# ----------------------------------------------------------------------------- selective recompute
+
+RECOMPUTE_CONFIG = "llama3_8b_l32"
+
+
+def recompute_work(w, n_tok, n_cow):
+    """Algorithmic FLOPs and bytes of the recompute, per layer."""
+    hk, d, dm = w.num_kv_heads, w.head_dim, w.d_model
+    n_out = 2 * hk * d                                         # K and V columns
+    gemm_flops = 2 * n_tok * dm * n_out
+    gemm_bytes = n_tok * dm * 2 + n_out * dm * 2 + n_tok * n_out * 2
+    row_bytes = hk * d * 2                                     # one slot of one page, all KV heads, one tensor
+    copy_bytes = 2 * 2 * (n_cow * 16 - n_tok) * row_bytes      # read + write of the non-selected slots, K and V
+    return {"gemm_flops": gemm_flops, "gemm_bytes": gemm_bytes, "copy_bytes": copy_bytes}
+
+
+def run_recompute(args, w, device, do_cpu):
+    """Plan once, then every layer's page copy and K/V projection for the
+    selection the fused step made on the workload's selecting layer."""
+    import serving_prefill_b200 as sp
+    from serving_prefill_b200 import Batch, KVPool
+    from serving_prefill_b200.engine import PrefillEngine, write_chunks
+    from workloads import make_recompute_inputs
+    torch.cuda.set_device(device)
+    lay = make_layout(w)
+    L, li = w.num_layers, w.impact_layer_index
+    n_refs = lay.page_ids.numel()
+    pool = KVPool(L, lay.num_pages + n_refs, w.num_kv_heads, w.head_dim, dtype=w.torch_dtype, device=device)
+    batch = Batch(lay.req_chunk_off, lay.chunk_doc_off, lay.chunk_page_off, lay.page_ids, lay.q_off, device=device)
+    eng = PrefillEngine(pool, batch, w.num_q_heads, w.r, dtype=w.torch_dtype, device=device)
+    inp = make_layer_inputs(w, lay, li)
+    write_chunks(pool, li, [p.to(torch.int32).to(device) for p in lay.chunk_pages],
+                 [k.to(device) for k in inp.chunk_k], [v.to(device) for v in inp.chunk_v])
+    eng.attend(li, inp.q.to(device), inp.kq.to(device), inp.vq.to(device), with_impact=True)
+    eng.select()
+    torch.cuda.synchronize()
+    k_host = eng.k.cpu().tolist()
+    n_sel = sum(k_host)
+    plan = torch.empty(sp.rag_recompute_plan_size(batch, eng.k_cap) // 4, dtype=torch.int32, device=device)
+    free = torch.arange(lay.num_pages, lay.num_pages + n_refs, dtype=torch.int32, device=device)
+    page_out = torch.empty_like(batch.dev[3])
+    rin = [make_recompute_inputs(w, lay, layer, rows=n_sel) for layer in range(L)]
+    xs = [r.x.to(device) for r in rin]
+    wks = [r.w_k.to(device) for r in rin]
+    wvs = [r.w_v.to(device) for r in rin]
+
+    def step():
+        sp.rag_recompute_plan(batch, eng.topk_idx, eng.k_cap, eng.k, free, page_out, plan, x_by_selection=True)
+        for layer in range(L):
+            sp.rag_recompute_kv(pool, layer, batch, eng.k_cap, plan, xs[layer], wks[layer], wvs[layer])
+
+    step()
+    torch.cuda.synchronize()
+    st, counts = sp.rag_recompute_status(plan)
+    if st != 0:
+        raise RuntimeError(f"recompute status {st}")
+    n_tok, n_cow, _ = counts
+    s_cap = torch.cuda.Stream()
+    s_cap.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s_cap):
+        step()
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(device)
+    clocks.start()
+    time.sleep(0.2)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        g.replay()
+    ev1.record()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    clk = clocks.stop()
+    # per-kernel device times: the step captured once more with event nodes
+    sp.rag_profile_collect()
+    sp.rag_profile_enable(True)
+    base = sp.rag_launch_count()
+    pg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(pg, stream=s_cap):
+        step()
+    launches = sp.rag_launch_count() - base
+    sp.rag_profile_enable(False)
+    torch.cuda.synchronize()
+    reps = max(3, min(args.steps, 50))
+    acc = {}
+    for _ in range(reps):
+        pg.replay()
+        torch.cuda.synchronize()
+        for kk, (m_k, c_k) in sp.rag_profile_peek().items():
+            a = acc.setdefault(kk, [0.0, 0])
+            a[0] += m_k
+            a[1] += c_k
+    sp.rag_profile_collect()
+    del pg, g
+    kinds = {kk: v for kk, v in acc.items() if v[1] > 0}
+    work = recompute_work(w, n_tok, n_cow)
+    peaks = load_peaks()
+    tflops_peak = peaks["bf16_tflops_sustained"] if ms > 1000.0 else peaks["bf16_tflops"]
+    per_launch = {"rc_gemm": (work["gemm_flops"], work["gemm_bytes"]), "rc_copy": (0, work["copy_bytes"])}
+    dom = max((kk for kk in kinds if kk in per_launch), key=lambda kk: kinds[kk][0])
+    avg_s = kinds[dom][0] / kinds[dom][1] / 1e3
+    flops, nbytes = per_launch[dom]
+    if flops:
+        ach = flops / avg_s / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": tflops_peak, "unit": "TFLOP/s", "frac": ach / tflops_peak}
+    else:
+        ach = nbytes / avg_s / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+    roof.update({"kernel": dom, "peak_source": peaks["source"], "avg_launch_us": avg_s * 1e6,
+                 "traffic": recorded_traffic("recompute_" + w.name, dom)})
+    ms_step = ms / args.steps
+    t_roof = max(L * work["gemm_flops"] / (tflops_peak * 1e12),
+                 L * (work["gemm_bytes"] + work["copy_bytes"]) / (peaks["hbm_gbs"] * 1e9))
+    # end to end through the C ABI: every layer's selected hidden states from pinned host memory,
+    # the rewritten page table back to the host
+    host_x = [r.x.pin_memory() for r in rin]
+    host_pages = torch.empty(page_out.numel(), dtype=torch.int32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        sp.rag_recompute_plan(batch, eng.topk_idx, eng.k_cap, eng.k, free, page_out, plan, x_by_selection=True)
+        for layer in range(L):
+            xs[layer].copy_(host_x[layer], non_blocking=True)
+            sp.rag_recompute_kv(pool, layer, batch, eng.k_cap, plan, xs[layer], wks[layer], wvs[layer])
+        host_pages.copy_(page_out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ev0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record()
+    torch.cuda.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
+    entry = {
+        "metric": "selected tokens/s through copy-on-write plan + page copy + K/V projection, all layers",
+        "value": n_tok / (ms_step / 1e3), "unit": "recomputed tokens/s", "ms_per_step": ms_step,
+        "config": {"workload": "recompute_" + w.name, "layers": L, "selected_tokens": n_tok,
+                   "private_pages": n_cow, "d_model": w.d_model, "kv_heads": w.num_kv_heads,
+                   "selection": "the fused step's top-k on the selecting layer (r = %g)" % w.r,
+                   "l2": "per-layer hidden states and weights (%.0f MB in all) exceed L2" %
+                         (sum(t.numel() * 2 for t in xs + wks + wvs) / 1e6),
+                   "timing": "CUDA graph replay per step"},
+        "roofline": roof, "step_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_step * 1e3,
+                                            "frac": t_roof / (ms_step / 1e3)},
+        "e2e": {"value": n_tok / (e2e_ms / 1e3), "unit": "recomputed tokens/s",
+                "h2d_bytes_per_step": sum(t.numel() * 2 for t in host_x), "d2h_bytes_per_step": page_out.numel() * 4},
+        "gpu_launches": int(launches * args.steps), "clocks": clk,
+        "kernels": {kk: {"ms_per_step": v[0] / reps, "launches_per_step": v[1] / reps} for kk, v in kinds.items()},
+        "work_per_layer": work,
+    }
+    if do_cpu:
+        entry["cpu_baseline"] = recompute_cpu_baseline(w, lay, eng.topk_idx.cpu(), k_host, rin, budget=5.0)
+    return entry
+
+
+def recompute_cpu_baseline(w, lay, topk_idx, k_host, rin, budget):
+    """The recompute oracle (plan + copy + projection) on the host cores over a sample of layers."""
+    import oracle.prefill as orc
+    import oracle.recompute as orc_rc
+    sel = [topk_idx[b, :k_host[b]].tolist() for b in range(len(k_host))]
+    n_refs = lay.page_ids.numel()
+    free = np.arange(lay.num_pages, lay.num_pages + n_refs)
+    pk = np.zeros((1, lay.num_pages + n_refs, w.num_kv_heads, 16, w.head_dim), dtype=np.uint16)
+    pv = pk.copy()
+    t0 = time.perf_counter()
+    p = orc_rc.plan(lay.req_chunk_off, lay.chunk_doc_off, lay.chunk_page_off, lay.page_ids, sel, free,
+                    x_by_selection=True)
+    t_plan = time.perf_counter() - t0
+    done, t_layers = 0, 0.0
+    while done < w.num_layers and t_layers < budget:
+        r = rin[done]
+        t0 = time.perf_counter()
+        orc_rc.apply(pk, pv, 0, p, orc.to_f64(r.x), orc.to_f64(r.w_k), orc.to_f64(r.w_v))
+        t_layers += time.perf_counter() - t0
+        done += 1
+    t_step = t_plan + t_layers * w.num_layers / done
+    return {"value": len(p.x_row) / t_step, "unit": "recomputed tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"plan once, then {done} of {w.num_layers} layers of copy + projection, "
+                      f"scaled to all layers; {t_step:.2f} s per step"}
+
+
+# ----------------------------------------------------------------------------- KV decode into the pool
+
+DECODE_CONFIG = "llama3_8b_l32"
+
+
+def decode_bits(w, layer):
+    """Compression level per part of the cache: 8 bits for the first half of the layers, 4 for the rest."""
+    return 8 if layer < w.num_layers // 2 else 4
+
+
+def run_kv_decode(args, w, device, do_cpu):
+    """Every layer of every distinct chunk decoded from its quantized stream into the pool."""
+    import serving_prefill_b200 as sp
+    from serving_prefill_b200 import KVPool
+    from workloads import make_encoded_layer
+    torch.cuda.set_device(device)
+    lay = make_layout(w)
+    L = w.num_layers
+    pool = KVPool(L, lay.num_pages, w.num_kv_heads, w.head_dim, dtype=w.torch_dtype, device=device)
+    n = list(lay.chunk_len)
+    tok_off = torch.tensor(np.cumsum([0] + n), dtype=torch.int32, device=device)
+    page_off = torch.tensor(np.cumsum([0] + [len(p) for p in lay.chunk_pages]), dtype=torch.int32, device=device)
+    pages = torch.cat(lay.chunk_pages).to(torch.int32).to(device)
+    enc = [make_encoded_layer(w, lay, layer, decode_bits(w, layer)) for layer in range(L)]
+    dev = [tuple(t.to(device) for t in (e.codes_k, e.codes_v, e.scale_k, e.offset_k, e.scale_v, e.offset_v))
+           for e in enc]
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def step(inputs):
+        for layer in range(L):
+            sp.rag_kv_decode(pool, layer, tok_off, page_off, pages, enc[layer].bits, *inputs[layer], device_err=err)
+
+    step(dev)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"kv decode device error {int(err.item())}")
+    s_cap = torch.cuda.Stream()
+    s_cap.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s_cap):
+        step(dev)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(device)
+    clocks.start()
+    time.sleep(0.2)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        g.replay()
+    ev1.record()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    clk = clocks.stop()
+    sp.rag_profile_collect()
+    sp.rag_profile_enable(True)
+    base = sp.rag_launch_count()
+    pg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(pg, stream=s_cap):
+        step(dev)
+    launches = sp.rag_launch_count() - base
+    sp.rag_profile_enable(False)
+    torch.cuda.synchronize()
+    reps = max(3, min(args.steps, 50))
+    tot, cnt = 0.0, 0
+    for _ in range(reps):
+        pg.replay()
+        torch.cuda.synchronize()
+        m_k, c_k = sp.rag_profile_peek()["kv_decode"]
+        tot += m_k
+        cnt += c_k
+    sp.rag_profile_collect()
+    del pg, g
+    # algorithmic bytes: codes and scales read, pages written (every slot of every page, K and V)
+    n_tok = sum(n)
+    n_pages = pages.numel()
+    hk, d = w.num_kv_heads, w.head_dim
+    per_layer = [2 * n_tok * hk * d * decode_bits(w, l) // 8 + 4 * len(n) * hk * d * 4 +
+                 2 * n_pages * hk * 16 * d * 2 for l in range(L)]
+    peaks = load_peaks()
+    avg_s = tot / cnt / 1e3
+    ach = (sum(per_layer) / L) / avg_s / 1e9
+    ms_step = ms / args.steps
+    t_roof = sum(per_layer) / (peaks["hbm_gbs"] * 1e9)
+    roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+            "kernel": "kv_decode", "peak_source": peaks["source"], "avg_launch_us": avg_s * 1e6,
+            "traffic": recorded_traffic("kv_decode_" + w.name, "kv_decode")}
+    # end to end: the compressed stream of every layer from pinned host memory, then decode
+    host = [tuple(t.pin_memory() for t in (e.codes_k, e.codes_v, e.scale_k, e.offset_k, e.scale_v, e.offset_v))
+            for e in enc]
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for layer in range(L):
+            for dt, ht in zip(dev[layer], host[layer]):
+                dt.copy_(ht, non_blocking=True)
+        step(dev)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ev0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record()
+    torch.cuda.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for trip in host for t in trip)
+    entry = {
+        "metric": "chunk KV tokens/s decoded from quantized streams into the pool, all layers",
+        "value": n_tok / (ms_step / 1e3), "unit": "decoded tokens/s (all layers)", "ms_per_step": ms_step,
+        "config": {"workload": "kv_decode_" + w.name, "layers": L, "chunks": len(n), "tokens": n_tok,
+                   "bits": "8 for layers 0-%d, 4 for layers %d-%d" % (L // 2 - 1, L // 2, L - 1),
+                   "l2": "codes of all layers (%.0f MB) and pages (%.0f MB) exceed L2" %
+                         (sum(e.codes_k.numel() * 2 for e in enc) / 1e6, pool.k.numel() * 4 / 1e6),
+                   "timing": "CUDA graph replay per step"},
+        "roofline": roof, "step_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": ms_step * 1e3,
+                                            "frac": t_roof / (ms_step / 1e3)},
+        "e2e": {"value": n_tok / (e2e_ms / 1e3), "unit": "decoded tokens/s (all layers)", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": int(launches * args.steps), "clocks": clk,
+        "kernels": {"kv_decode": {"ms_per_step": tot / reps, "launches_per_step": cnt / reps}},
+    }
+    if do_cpu:
+        entry["cpu_baseline"] = kv_decode_cpu_baseline(w, lay, enc, budget=3.0)
+    return entry
+
+
+def kv_decode_cpu_baseline(w, lay, enc, budget):
+    """The codec oracle decoding a sample of layers into a host pool."""
+    import oracle.codec as codec
+    pk = np.zeros((1, lay.num_pages, w.num_kv_heads, 16, w.head_dim), dtype=np.uint16)
+    pv = pk.copy()
+    done, t = 0, 0.0
+    tok0 = np.cumsum([0] + list(lay.chunk_len))
+    while done < w.num_layers and t < budget:
+        e = enc[done]
+        t0 = time.perf_counter()
+        for c, pages in enumerate(lay.chunk_pages):
+            a, b = tok0[c], tok0[c + 1]
+            ch = codec.EncodedChunk(e.bits, e.codes_k[a:b].numpy(), e.codes_v[a:b].numpy(), e.scale_k[c].numpy(),
+                                    e.offset_k[c].numpy(), e.scale_v[c].numpy(), e.offset_v[c].numpy())
+            codec.decode_into_pool(pk, pv, 0, pages.numpy(), ch, lay.chunk_len[c])
+        t += time.perf_counter() - t0
+        done += 1
+    t_step = t * w.num_layers / done
+    return {"value": sum(lay.chunk_len) / t_step, "unit": "decoded tokens/s (all layers)", "cores": blas_threads(),
+            "kind": "oracle", "sample": f"{done} of {w.num_layers} layers, scaled to all; {t_step:.2f} s per step"}
+
+
 # ----------------------------------------------------------------------------- CPU oracle arm
 
 def blas_threads():
@@ -615,6 +954,12 @@ def main():
                      "cpu_baseline": cpu_baseline(wc, 2.0) if do_cpu else None, "e2e": rc["e2e"],
                      "gpu_launches": rc["gpu_launches"], "clocks": rc["clocks"], "kernels": rc["kernels"]}
             per_config[name] = entry
+        wr = get_workload(RECOMPUTE_CONFIG)
+        per_config["recompute_" + wr.name] = run_recompute(args, wr, device, do_cpu)
+        torch.cuda.empty_cache()
+        wd = get_workload(DECODE_CONFIG)
+        per_config["kv_decode_" + wd.name] = run_kv_decode(args, wd, device, do_cpu)
+        torch.cuda.empty_cache()
 
     if rank == 0:
         line = {

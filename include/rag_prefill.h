@@ -250,6 +250,35 @@ RAG_API int32_t rag_recompute_count(int32_t n_doc, double r);
 RAG_API rag_status rag_impact_topk(const float* impact, const rag_batch* batch, double r, int32_t k_cap,
                            int32_t* topk_idx, float* topk_val, int32_t* k_out, void* stream);
 
+/* ---- Decode of quantized chunk caches into the pool ---------------------------
+ * CacheGen page, "How the technology works": a prefilled chunk's KV cache is
+ * kept (or sent) as a compact stream and decoded on the GPU into a KV cache
+ * from which generation starts; its glossary names quantization with
+ * different compression levels for different parts of the cache. The pages
+ * give no stream format; this entry point decodes the plainest one they
+ * support: per chunk, layer, KV head and channel, b-bit codes (b = 8 or 4,
+ * chosen per call, i.e. per layer) of a uniform quantization with an fp32
+ * scale and offset. value = fp32 fma(code, scale, offset), stored as bf16.
+ *
+ * One call decodes n_chunks chunks of one layer (bf16 pool, head_dim 128):
+ *   chunk_tok_off  [n_chunks+1] device int32: token prefix over the chunks
+ *   chunk_page_off [n_chunks+1] device int32: page prefix; chunk c owns
+ *                  ceil(n_c / 16) pages
+ *   page_ids       [total_pages] device int32: destination pages, in order
+ *   codes_k/v      [total_tokens][num_kv_heads][128 * bits / 8] device bytes,
+ *                  8-byte aligned (4 bits: even channel in the low nibble)
+ *   scale_k/v, offset_k/v [n_chunks][num_kv_heads][128] device fp32, 16-byte
+ *                  aligned
+ * Token t of chunk c lands in slot t % 16 of page page_ids[chunk_page_off[c] +
+ * t / 16]; the last page's slots past the chunk are zeroed. A page id outside
+ * the pool or a chunk whose page count is not ceil(n_c / 16) is skipped and
+ * recorded in *device_err (optional device int32: 1 page, 2 geometry). */
+RAG_API rag_status rag_kv_decode(const rag_kv_pool* pool, int32_t layer, int32_t n_chunks,
+                                 const int32_t* chunk_tok_off, const int32_t* chunk_page_off,
+                                 const int32_t* page_ids, int32_t total_pages, int32_t bits, const void* codes_k,
+                                 const void* codes_v, const float* scale_k, const float* offset_k,
+                                 const float* scale_v, const float* offset_v, int32_t* device_err, void* stream);
+
 /* ---- Selective recompute of the chosen tokens' K and V ---------------------
  * CacheBlend page, "Contributions" (only the tokens of high attention impact
  * are recomputed when the cached KV are fused) and "How it works" (after the
@@ -340,7 +369,7 @@ RAG_API int64_t rag_launch_count(void);
  * milliseconds and launch counts per kernel kind (0 pool write, 1 attention,
  * 2 split combine, 3 impact, 4 top-k, 5 fp32 attention, 6 fp32 impact,
  * 7 recompute plan, 8 recompute page copy, 9 recompute projection,
- * 10 RoPE table) into
+ * 10 RoPE table, 11 KV decode) into
  * the first n_kinds entries of ms and launches (either may be NULL), and
  * resets the record. */
 RAG_API void rag_profile_enable(int32_t on);

@@ -16,6 +16,7 @@ from .rag import (  # noqa: F401
     rag_fused_prefill_attn,
     rag_fused_prefill_attn_rope,
     rag_impact_topk,
+    rag_kv_decode,
     rag_kv_pool_write,
     rag_last_device_error,
     rag_launch_count,

@@ -54,11 +54,14 @@ struct TileDesc {
 
 struct FwdCtrl {
   uint64_t q_full, q_empty;
-  uint64_t kfull[kKStages], kempty[kKStages];
+  uint64_t kfull[kKStages], kempty[kKStages], kconv[kKStages];
   uint64_t vfull[kVStages], vempty[kVStages], vconv[kVStages];
-  // s_full[b] / p_full[b]: S buffer b (Q tile b's columns; with one Q tile in
-  // the item, both buffers serve Q tile 0 in turn)
-  uint64_t s_full[kQTiles], p_full[kQTiles], pv_done[kQTiles], o_full[kQTiles], o_free[kQTiles];
+  int32_t kchunk[kKStages][kPagesPerTile];   // chunk-list entry per page of a K stage (-1: none)
+  // s_full[b] / p_lo[b] / p_hi[b]: S buffer b (Q tile b's columns; with one Q
+  // tile in the item, both buffers serve Q tile 0 in turn); P of keys 0-63 and
+  // of keys 64-127 are published separately, so that PV over the first half
+  // runs while the second half is exponentiated
+  uint64_t s_full[kQTiles], p_lo[kQTiles], p_hi[kQTiles], pv_done[kQTiles], o_full[kQTiles], o_free[kQTiles];
   uint64_t teardown;
   uint64_t desc_full[kDescSlots], desc_empty[kDescSlots];
   TileDesc desc[kDescSlots];
@@ -158,7 +161,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (tid == 0) {
     mbar_init(&ctl->q_full, 1);
     mbar_init(&ctl->q_empty, 1);
-    for (int s = 0; s < kKStages; ++s) { mbar_init(&ctl->kfull[s], 1); mbar_init(&ctl->kempty[s], 1); }
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&ctl->kfull[s], 1);
+      mbar_init(&ctl->kempty[s], 1);
+      mbar_init(&ctl->kconv[s], 1);
+    }
     for (int s = 0; s < kVStages; ++s) {
       mbar_init(&ctl->vfull[s], 1);
       mbar_init(&ctl->vempty[s], 1);
@@ -166,7 +173,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int q = 0; q < kQTiles; ++q) {
       mbar_init(&ctl->s_full[q], 1);
-      mbar_init(&ctl->p_full[q], 128);
+      mbar_init(&ctl->p_lo[q], 128);
+      mbar_init(&ctl->p_hi[q], 128);
       mbar_init(&ctl->pv_done[q], 1);
       mbar_init(&ctl->o_full[q], 1);
       mbar_init(&ctl->o_free[q], 128);
@@ -286,24 +294,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!mbar_wait(&ctl->s_full[sb], (sb ? n_sf1 : n_sf0) & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
         if (!warp_live) {
-          mbar_arrive(&ctl->p_full[sb]);
+          mbar_arrive(&ctl->p_lo[sb]);
+          mbar_arrive(&ctl->p_hi[sb]);
           if (sb) ++n_sf1; else ++n_sf0;
           ++n_pvq;
           continue;
         }
         float x[kBN];
         {
-          uint32_t u0[32], u1[32];
+          // the whole row in one round trip: four loads, one wait
+          uint32_t u0[32], u1[32], u2[32], u3[32];
           tmem_ld32(s_addr + 0, u0);
           tmem_ld32(s_addr + 32, u1);
+          tmem_ld32(s_addr + 64, u2);
+          tmem_ld32(s_addr + 96, u3);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) { x[j] = __uint_as_float(u0[j]); x[32 + j] = __uint_as_float(u1[j]); }
-          tmem_ld32(s_addr + 64, u0);
-          tmem_ld32(s_addr + 96, u1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) { x[64 + j] = __uint_as_float(u0[j]); x[96 + j] = __uint_as_float(u1[j]); }
+          for (int j = 0; j < 32; ++j) {
+            x[j] = __uint_as_float(u0[j]);
+            x[32 + j] = __uint_as_float(u1[j]);
+            x[64 + j] = __uint_as_float(u2[j]);
+            x[96 + j] = __uint_as_float(u3[j]);
+          }
         }
         // mask (only partial tiles), then the row max of the raw scores
         if (td.kind == 0) {
@@ -381,12 +393,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             pk[j] = pack_f16x2(e.x, e.y);
           }
           tmem_st32(s_addr + 32 * h, pk);   // P over the first 64 columns of S
+          // publish this half of P: PV over its 64 keys may start
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(h == 0 ? &ctl->p_lo[sb] : &ctl->p_hi[sb]);
         }
         const float2 ls01 = fadd2(ls[0], ls[1]), ls23 = fadd2(ls[2], ls[3]);
         l_sum += (ls01.x + ls01.y) + (ls23.x + ls23.y);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&ctl->p_full[sb]);
         if (sb) ++n_sf1; else ++n_sf0;
         ++n_pvq;
       }
@@ -547,6 +560,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           bad = 1;
           break;
         }
+        if (is_k && lane < kPagesPerTile) ctl->kchunk[s][lane] = (doc && pg.page >= 0) ? pg.chunk : -1;
+        __syncwarp();
         if (lane == 0) mbar_arrive_expect_tx(&full[s], kTileBytes);
         __syncwarp();
         uint8_t* dst = sbase + s * kTileBytes;
@@ -590,6 +605,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int n = it.t_end - it.t_begin;
       for (int i = 0; i < n; ++i) {
         const uint32_t t = t_glob + i;
+        if (p.rope) {
+          // re-base the cached keys of this K tile to their concatenated positions
+          const int sk = t % kKStages;
+          if (!mbar_wait(&ctl->kfull[sk], (t / kKStages) & 1, abort_flag)) { bad = 1; break; }
+          rope_rotate_tile(sK + sk * kTileBytes, ctl->kchunk[sk], p.rope, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->kconv[sk]);
+        }
         const int s = t % kVStages;
         if (!mbar_wait(&ctl->vfull[s], (t / kVStages) & 1, abort_flag)) { bad = 1; break; }
         uint4* tile = reinterpret_cast<uint4*>(sV + s * kTileBytes);
@@ -622,7 +646,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t idesc_pv = idesc_f16_f32(kBM, kHeadDim, 1);
       const uint32_t q_base = smem_u32(sQ);
       uint32_t t_glob = 0, q_iter = 0;
-      uint32_t n_pf0 = 0, n_pf1 = 0;       // completions of p_full[0] / p_full[1] consumed
+      uint32_t n_pf0 = 0, n_pf1 = 0;       // completions of p_lo/p_hi[0] and [1] consumed
       uint32_t n_item[kQTiles] = {0, 0};   // items begun, per Q tile
       int bad = 0;
       for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
@@ -638,7 +662,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           auto qk = [&](int j) {
             const uint32_t t = t_glob + j;
             const int s = t % kKStages;
-            if (!mbar_wait(&ctl->kfull[s], (t / kKStages) & 1, abort_flag)) return false;
+            if (!mbar_wait(p.rope ? &ctl->kconv[s] : &ctl->kfull[s], (t / kKStages) & 1, abort_flag)) return false;
             const uint32_t k_base = smem_u32(sK + s * kTileBytes);
             tc_fence_after();
 #pragma unroll
@@ -661,13 +685,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               ++n_item[0];
             }
             uint32_t& npf = b ? n_pf1 : n_pf0;
-            if (!mbar_wait(&ctl->p_full[b], npf & 1, abort_flag)) { bad = 1; break; }
-            ++npf;
-            tc_fence_after();
             const uint32_t v_base = smem_u32(sV + sv * kTileBytes);
+            bool ok = true;
+            for (int hh = 0; hh < 2 && ok; ++hh) {
+              if (!mbar_wait(hh == 0 ? &ctl->p_lo[b] : &ctl->p_hi[b], npf & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
-              mma_ts(tmem + col_o(0), tmem + col_s(b) + kk * 8, v_desc(v_base, kk), idesc_pv, (i > 0) || (kk > 0));
+              for (int kk = 4 * hh; kk < 4 * hh + 4; ++kk)
+                mma_ts(tmem + col_o(0), tmem + col_s(b) + kk * 8, v_desc(v_base, kk), idesc_pv, (i > 0) || (kk > 0));
+            }
+            if (!ok) { bad = 1; break; }
+            ++npf;
             tc_commit(&ctl->pv_done[0]);
             if (i == n - 1) tc_commit(&ctl->o_full[0]);
             tc_commit(&ctl->vempty[sv]);
@@ -691,7 +719,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             v_base = smem_u32(sV + sv * kTileBytes);
           }
           if (i < n) {
-            if (!mbar_wait(&ctl->kfull[s], (t / kKStages) & 1, abort_flag)) { bad = 1; break; }
+            if (!mbar_wait(p.rope ? &ctl->kconv[s] : &ctl->kfull[s], (t / kKStages) & 1, abort_flag)) {
+              bad = 1;
+              break;
+            }
             k_base = smem_u32(sK + s * kTileBytes);
           }
           for (int q = 0; q < it.n_qt && !bad; ++q) {
@@ -705,13 +736,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ++n_item[q];
               }
               uint32_t& npf = q ? n_pf1 : n_pf0;
-              if (!mbar_wait(&ctl->p_full[q], npf & 1, abort_flag)) { bad = 1; break; }
-              ++npf;
-              tc_fence_after();
+              bool ok = true;
+              for (int hh = 0; hh < 2 && ok; ++hh) {
+                if (!mbar_wait(hh == 0 ? &ctl->p_lo[q] : &ctl->p_hi[q], npf & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
-              for (int kk = 0; kk < kBN / 16; ++kk)
-                mma_ts(tmem + col_o(q), tmem + col_s(q) + kk * 8, v_desc(v_base, kk), idesc_pv,
-                       (i > 1) || (kk > 0));
+                for (int kk = 4 * hh; kk < 4 * hh + 4; ++kk)
+                  mma_ts(tmem + col_o(q), tmem + col_s(q) + kk * 8, v_desc(v_base, kk), idesc_pv,
+                         (i > 1) || (kk > 0));
+              }
+              if (!ok) { bad = 1; break; }
+              ++npf;
               tc_commit(&ctl->pv_done[q]);
               if (i == n) tc_commit(&ctl->o_full[q]);   // O_q of this item is complete
             }
@@ -838,7 +873,34 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p
   }
 }
 
+// ---------------------------------------------------------------- RoPE table
+
+// Per chunk-list entry e of request b, the re-basing angle of every rotary
+// pair: offset o_e (doc tokens of the request before the entry) times
+// theta_i = base^(-2 i / 128), as (cos, sin), computed in fp64 and stored in
+// fp32. One block per request.
+__global__ void __launch_bounds__(256) rope_table_kernel(const BatchDev B, double base, float2* table) {
+  pdl_launch_dependents();
+  const ReqInfo r = load_req(B, blockIdx.x);
+  if (!req_ok(B, r)) return;
+  pdl_wait();   // the kernel before this one may still read the table of the previous call
+  const int n = (r.c1 - r.c0) * 64;
+  for (int idx = threadIdx.x; idx < n; idx += blockDim.x) {
+    const int e = r.c0 + idx / 64, i = idx % 64;
+    const double o = double(__ldg(B.chunk_doc_off + e) - r.doc0);
+    const double theta = pow(base, -2.0 * double(i) / double(kHeadDim));
+    double sn, cn;
+    sincos(o * theta, &sn, &cn);
+    table[int64_t(e) * 64 + i] = make_float2(float(cn), float(sn));
+  }
+}
+
 // ---------------------------------------------------------------- launchers
+
+cudaError_t launch_rope_table(const BatchDev& b, double base, float2* table, cudaStream_t stream) {
+  return launch_pdl(rope_table_kernel, dim3(b.num_requests), dim3(256), 0, stream, 1, b, base, table);
+}
+
 
 cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tkq, const CUtensorMap& tvq, const FwdParams& p, int grid,

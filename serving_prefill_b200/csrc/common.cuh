@@ -115,12 +115,13 @@ struct PageRef {
   int32_t page;     // physical page, or -1 when absent/invalid
   int32_t nvalid;   // valid slots (0..16)
   int32_t lstart;   // logical doc position of slot 0 within the request
+  int32_t chunk;    // chunk-list entry the page belongs to (-1 when absent)
 };
 
 __device__ __forceinline__ PageRef page_ref(const BatchDev& B, const ReqInfo& r, int ref, int num_pages,
                                             int32_t* err) {
   PageRef p;
-  p.page = -1; p.nvalid = 0; p.lstart = 0;
+  p.page = -1; p.nvalid = 0; p.lstart = 0; p.chunk = -1;
   if (ref >= r.n_pages) return p;
   const int gref = r.p0 + ref;
   const int c = chunk_of_page(B, r.c0, r.c1, gref);
@@ -145,6 +146,7 @@ __device__ __forceinline__ PageRef page_ref(const BatchDev& B, const ReqInfo& r,
   p.page = page;
   p.nvalid = nv;
   p.lstart = cstart - r.doc0 + k * kPage;
+  p.chunk = c;
   return p;
 }
 
@@ -180,7 +182,7 @@ __device__ __forceinline__ PageRef page_ref_cached(const ChunkCache* cc, const B
                                                    int ref, int32_t page, int num_pages, int32_t* err) {
   if (cc->n < 0) return page_ref(B, r, ref, num_pages, err);
   PageRef p;
-  p.page = -1; p.nvalid = 0; p.lstart = 0;
+  p.page = -1; p.nvalid = 0; p.lstart = 0; p.chunk = -1;
   if (ref >= r.n_pages) return p;
   const int gref = r.p0 + ref;
   int lo = 0, hi = cc->n - 1;   // last local chunk with page_off <= gref
@@ -208,7 +210,57 @@ __device__ __forceinline__ PageRef page_ref_cached(const ChunkCache* cc, const B
   p.page = page;
   p.nvalid = nv;
   p.lstart = cstart - r.doc0 + k * kPage;
+  p.chunk = r.c0 + lo;
   return p;
+}
+
+// RoPE re-basing of one K tile in shared memory (TurboRAG page,
+// "Implementation": position ids of precompute and inference must agree).
+// The tile is 128 keys x 128 channels of bf16, stored as two 64-channel
+// halves (16 KB apart), each 128B-swizzled: the 16-byte column c of row r
+// sits at r * 128 + ((c ^ (r & 7)) * 16) in both halves, so one 16-byte load
+// from each half holds the 8 rotary pairs (i, i + 64), i = 8c .. 8c + 7.
+// Key r belongs to page r / 16 of the tile, whose chunk-list entry is
+// kchunk[r / 16] (-1: not a cached key, left alone); pair i of entry e turns
+// by the angle in table[e * 64 + i] = (cos, sin). Each pair is rotated in
+// fp32 and rounded once to bf16. One warp, every lane on one column c.
+__device__ __forceinline__ void rope_rotate_tile(uint8_t* tile, const int32_t* kchunk, const float2* table,
+                                                 int lane) {
+  const int c = lane & 7;
+  int cur = -1;
+  float2 cs[8];
+#pragma unroll 1
+  for (int r = lane >> 3; r < 128; r += 4) {
+    const int e = kchunk[r >> 4];
+    if (e < 0) continue;
+    if (e != cur) {
+      const float4* t4 = reinterpret_cast<const float4*>(table + int64_t(e) * 64 + c * 8);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 v = __ldg(t4 + j);
+        cs[2 * j] = make_float2(v.x, v.y);
+        cs[2 * j + 1] = make_float2(v.z, v.w);
+      }
+      cur = e;
+    }
+    uint4* p0 = reinterpret_cast<uint4*>(tile + r * 128 + ((c ^ (r & 7)) << 4));
+    uint4* p1 = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p0) + 16384);
+    uint4 a = *p0, b = *p1;
+    uint32_t* aw = reinterpret_cast<uint32_t*>(&a);
+    uint32_t* bw = reinterpret_cast<uint32_t*>(&b);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float x0 = __uint_as_float(aw[w] << 16), x1 = __uint_as_float(aw[w] & 0xffff0000u);
+      const float y0 = __uint_as_float(bw[w] << 16), y1 = __uint_as_float(bw[w] & 0xffff0000u);
+      const float2 c0 = cs[2 * w], c1 = cs[2 * w + 1];
+      const float nx0 = fmaf(x0, c0.x, -(y0 * c0.y)), ny0 = fmaf(y0, c0.x, x0 * c0.y);
+      const float nx1 = fmaf(x1, c1.x, -(y1 * c1.y)), ny1 = fmaf(y1, c1.x, x1 * c1.y);
+      aw[w] = pack_bf16x2(nx0, nx1);
+      bw[w] = pack_bf16x2(ny0, ny1);
+    }
+    *p0 = a;
+    *p1 = b;
+  }
 }
 
 // Workspace layout (bytes, each region 256-aligned):
@@ -217,19 +269,22 @@ __device__ __forceinline__ PageRef page_ref_cached(const ChunkCache* cc, const B
 //   row_m2                     total_q * H_q fp32   (reference max, log2 units)
 //   row_il                     total_q * H_q fp32   (1 / (l * H_q))
 //   partials                   items * 256 * kPartStride 32-bit words
+//   RoPE table                 num_chunks * 64 (cos, sin) fp32 pairs
 struct WsLayout {
-  size_t off_prefix, off_m2, off_il, off_part, total;
+  size_t off_prefix, off_m2, off_il, off_part, off_rope, total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-__host__ __device__ inline WsLayout ws_layout(int64_t total_q, int num_q_heads, int64_t max_items) {
+__host__ __device__ inline WsLayout ws_layout(int64_t total_q, int num_q_heads, int64_t max_items,
+                                              int64_t num_chunks) {
   WsLayout w;
   size_t at = 256;
   w.off_prefix = at; at = align256(at + sizeof(int32_t) * (kMaxRequests + 1));
   w.off_m2 = at; at = align256(at + sizeof(float) * size_t(total_q) * num_q_heads);
   w.off_il = at; at = align256(at + sizeof(float) * size_t(total_q) * num_q_heads);
   w.off_part = at; at = align256(at + sizeof(float) * size_t(max_items) * kFwdRows * kPartStride);
+  w.off_rope = at; at = align256(at + sizeof(float) * 2 * 64 * size_t(num_chunks));
   w.total = at;
   return w;
 }

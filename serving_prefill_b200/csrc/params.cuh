@@ -198,6 +198,23 @@ struct RcGemmParams {
   int64_t max_tok;
 };
 
+struct KvDecodeParams {
+  __nv_bfloat16* pool_k;
+  __nv_bfloat16* pool_v;
+  const int32_t* chunk_tok_off;    // [n_chunks + 1]
+  const int32_t* chunk_page_off;   // [n_chunks + 1]
+  const int32_t* page_ids;         // [total pages]
+  const uint8_t* codes_k;
+  const uint8_t* codes_v;
+  const float* scale_k;
+  const float* offset_k;
+  const float* scale_v;
+  const float* offset_v;
+  int32_t* err;
+  int32_t layer, num_pages, num_kv_heads, n_chunks, bits;
+};
+cudaError_t launch_kv_decode(const KvDecodeParams&, int total_pages, cudaStream_t);
+
 cudaError_t launch_rc_plan(const RcPlanParams&, cudaStream_t);
 cudaError_t launch_rc_copy(const RcCopyParams&, int grid, cudaStream_t);
 cudaError_t launch_rc_gemm(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const RcGemmParams&, int grid,

@@ -24,7 +24,7 @@ constexpr int kRcMinDModel = 64;
 // ------------------------------------------------------------ profiling
 
 enum Kind { kKindPoolWrite = 0, kKindAttn, kKindCombine, kKindImpact, kKindTopk, kKindSimtAttn, kKindSimtImpact,
-            kKindRcPlan, kKindRcCopy, kKindRcGemm, kKindRope, kNumKinds };
+            kKindRcPlan, kKindRcCopy, kKindRcGemm, kKindRope, kKindKvDecode, kNumKinds };
 
 struct ProfRecord {
   int kind;
@@ -526,6 +526,51 @@ rag_status rag_impact_topk(const float* impact, const rag_batch* batch, double r
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   LaunchScope ls(kKindTopk, s);
   cudaError_t e = launch_topk(p, b.num_requests, p.k_max, s);
+  ls.done(e);
+  return e == cudaSuccess ? RAG_OK : RAG_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ KV decode into the pool
+
+rag_status rag_kv_decode(const rag_kv_pool* pool, int32_t layer, int32_t n_chunks, const int32_t* chunk_tok_off,
+                         const int32_t* chunk_page_off, const int32_t* page_ids, int32_t total_pages, int32_t bits,
+                         const void* codes_k, const void* codes_v, const float* scale_k, const float* offset_k,
+                         const float* scale_v, const float* offset_v, int32_t* device_err, void* stream) {
+  rag_status st = check_pool(pool);
+  if (st != RAG_OK) return st;
+  if (pool->dtype != RAG_BF16) return RAG_ERR_UNSUPPORTED;
+  if (layer < 0 || layer >= pool->num_layers) return RAG_ERR_INVALID_ARG;
+  if (bits != 4 && bits != 8) return RAG_ERR_UNSUPPORTED;
+  if (n_chunks < 0 || total_pages < 0) return RAG_ERR_SHAPE;
+  if (n_chunks == 0 || total_pages == 0) return RAG_OK;
+  if (!chunk_tok_off || !chunk_page_off || !page_ids || !codes_k || !codes_v || !scale_k || !offset_k ||
+      !scale_v || !offset_v)
+    return RAG_ERR_INVALID_ARG;
+  // codes: 8-byte (8-bit) or 4-byte (4-bit) loads per 8 channels; scales: 16-byte loads
+  if ((reinterpret_cast<uintptr_t>(codes_k) | reinterpret_cast<uintptr_t>(codes_v)) & 7u) return RAG_ERR_INVALID_ARG;
+  if (!aligned16(scale_k) || !aligned16(offset_k) || !aligned16(scale_v) || !aligned16(offset_v))
+    return RAG_ERR_INVALID_ARG;
+  KvDecodeParams p;
+  p.pool_k = static_cast<__nv_bfloat16*>(pool->k);
+  p.pool_v = static_cast<__nv_bfloat16*>(pool->v);
+  p.chunk_tok_off = chunk_tok_off;
+  p.chunk_page_off = chunk_page_off;
+  p.page_ids = page_ids;
+  p.codes_k = static_cast<const uint8_t*>(codes_k);
+  p.codes_v = static_cast<const uint8_t*>(codes_v);
+  p.scale_k = scale_k;
+  p.offset_k = offset_k;
+  p.scale_v = scale_v;
+  p.offset_v = offset_v;
+  p.err = device_err;
+  p.layer = layer;
+  p.num_pages = pool->num_pages;
+  p.num_kv_heads = pool->num_kv_heads;
+  p.n_chunks = n_chunks;
+  p.bits = bits;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  LaunchScope ls(kKindKvDecode, s);
+  cudaError_t e = launch_kv_decode(p, total_pages, s);
   ls.done(e);
   return e == cudaSuccess ? RAG_OK : RAG_ERR_CUDA;
 }

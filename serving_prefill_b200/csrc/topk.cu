@@ -29,8 +29,9 @@ constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkBins = 4096;
 constexpr int kBatch = 8;            // keys in flight per thread per pass
-constexpr int kTopkMaxK = 16384;     // largest k
+constexpr int kTopkMaxK = 16384;     // largest k (the host rejects more)
 constexpr int kTopkSortMax = 20480;  // staged keys: those above the k-th key's bucket, then its candidates
+static_assert(kTopkMaxK <= kTopkSortMax, "the k selected keys must fit the staging array");
 constexpr int kTopkMaxCluster = 8;
 constexpr int kTopkSlice = 8192;     // doc tokens per CTA before the cluster grows
 constexpr int kRankMax = 256;        // longest bucket ordered by counting ranks (longer: sorted)
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   const int csize = int(cluster.num_blocks());
   const int crank = int(cluster.block_rank());
   const int b = blockIdx.x / csize;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const ReqInfo req = load_req(p.batch, b);
   const bool ok = req_ok(p.batch, req);
   const int n = ok ? req.n_doc : 0;

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librag.so")
 RAG_BF16, RAG_F32 = 0, 1
 PAGE_SIZE = 16
 KERNEL_KINDS = ("pool_write", "attn", "combine", "impact", "topk", "simt_attn", "simt_impact", "rc_plan", "rc_copy",
-                "rc_gemm", "rope_table")
+                "rc_gemm", "rope_table", "kv_decode")
 
 STATUS = {
     0: "ok", 1: "invalid argument", 2: "inconsistent shape", 3: "page id outside the pool",
@@ -72,6 +72,8 @@ EXPORTS = {
                                   c_void_p]),
     "rag_last_device_error": (c_int32, [c_void_p, c_void_p, c_void_p]),
     "rag_selftest_wait_timeout": (c_int32, [c_void_p, c_int64, c_void_p]),
+    "rag_kv_decode": (c_int32, [POINTER(RagKVPool), c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int32, c_int32,
+                                c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "rag_recompute_plan_size": (c_size_t, [POINTER(RagBatch), c_int32]),
     "rag_recompute_plan": (c_int32, [POINTER(RagBatch), c_void_p, c_int32, c_void_p, c_void_p, c_int32, c_int32,
                                      c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -251,6 +253,16 @@ def rag_last_device_error(workspace: torch.Tensor, stream=None) -> tuple:
 def rag_selftest_wait_timeout(device_err: torch.Tensor, limit_ns: int, stream=None):
     _check(lib().rag_selftest_wait_timeout(_ptr(device_err), limit_ns, _stream(stream)),
            "rag_selftest_wait_timeout")
+
+
+def rag_kv_decode(pool: KVPool, layer: int, chunk_tok_off: torch.Tensor, chunk_page_off: torch.Tensor,
+                  page_ids: torch.Tensor, bits: int, codes_k: torch.Tensor, codes_v: torch.Tensor,
+                  scale_k: torch.Tensor, offset_k: torch.Tensor, scale_v: torch.Tensor, offset_v: torch.Tensor,
+                  device_err: torch.Tensor = None, stream=None):
+    _check(lib().rag_kv_decode(ctypes.byref(pool.c), layer, chunk_tok_off.numel() - 1, _ptr(chunk_tok_off),
+                               _ptr(chunk_page_off), _ptr(page_ids), page_ids.numel(), bits, _ptr(codes_k),
+                               _ptr(codes_v), _ptr(scale_k), _ptr(offset_k), _ptr(scale_v), _ptr(offset_v),
+                               _ptr(device_err), _stream(stream)), "rag_kv_decode")
 
 
 def rag_recompute_plan_size(batch: Batch, k_cap: int) -> int:

@@ -15,6 +15,7 @@ from .rag import (  # noqa: F401
     RecomputeInputs,
     make_recompute_inputs,
     random_selection,
+    make_encoded_layer,
     make_layout,
     make_layer_inputs,
     get_workload,

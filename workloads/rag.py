@@ -142,7 +142,7 @@ def _gen(seed: int, *tags: int) -> torch.Generator:
 
 
 # sub-stream tags
-_T_LAYOUT, _T_SCALE, _T_Q, _T_K, _T_V, _T_KQ, _T_VQ, _T_X, _T_WK, _T_WV = range(10)
+_T_LAYOUT, _T_SCALE, _T_Q, _T_K, _T_V, _T_KQ, _T_VQ, _T_X, _T_WK, _T_WV, _T_CODES = range(11)
 
 
 @dataclass
@@ -333,3 +333,28 @@ def random_selection(doc_lens, counts, seed: int) -> list:
         k = min(int(k), int(n))
         out.append(torch.randperm(int(n), generator=g)[:k].tolist() if n > 0 else [])
     return out
+
+
+@dataclass
+class EncodedLayer:
+    """A synthetic quantized stream of every distinct chunk of one layer: random
+    b-bit codes [total_tokens][H_kv][128 * b / 8] (bytes) for K and V, and per
+    chunk, KV head and channel an fp32 scale (lognormal) and offset (normal)."""
+    bits: int
+    codes_k: torch.Tensor
+    codes_v: torch.Tensor
+    scale_k: torch.Tensor
+    offset_k: torch.Tensor
+    scale_v: torch.Tensor
+    offset_v: torch.Tensor
+
+
+def make_encoded_layer(w: Workload, lay: BatchLayout, layer: int, bits: int) -> EncodedLayer:
+    g = _gen(w.seed, _T_CODES, layer)
+    n = sum(lay.chunk_len)
+    row = w.head_dim * bits // 8
+    nc = len(lay.chunk_len)
+    codes = lambda: torch.randint(0, 256, (n, w.num_kv_heads, row), generator=g, dtype=torch.int32).to(torch.uint8)
+    scale = lambda: torch.exp(0.5 * torch.randn(nc, w.num_kv_heads, w.head_dim, generator=g)) * 0.02
+    offset = lambda: -2.0 + 0.5 * torch.randn(nc, w.num_kv_heads, w.head_dim, generator=g)
+    return EncodedLayer(bits, codes(), codes(), scale(), offset(), scale(), offset())
