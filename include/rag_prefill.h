@@ -35,9 +35,14 @@
  *   - Indices of doc tokens are logical positions within their request,
  *     0 .. N_doc,b - 1, in concatenation order.
  *   - Stream order holds as usual. The kernels are launched with programmatic
- *     stream serialization: a kernel may begin its set-up (shared memory,
- *     tensor memory) while the previous kernel in the stream finishes, but it
- *     reads and writes global memory only after that kernel has completed.
+ *     stream serialization. When the previous kernel in the stream is one of
+ *     this library's attention, combine, Impact or top-k kernels, the next
+ *     one may start while it finishes: it sets up and reads its own inputs
+ *     (the pool, the batch descriptors, q, kq, vq), none of which those
+ *     kernels write, and writes global memory only after the previous kernel
+ *     has completed. Kernels that write pool pages, page tables or the RoPE
+ *     table (pool write, KV decode, recompute, RoPE table) and every kernel
+ *     not of this library let the next kernel start only when they complete.
  */
 #ifndef RAG_PREFILL_H_
 #define RAG_PREFILL_H_

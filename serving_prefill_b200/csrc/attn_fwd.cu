@@ -196,13 +196,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   }
   if (warp == 9 && lane == 0) { tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_vq); }
 
-  // Everything above touches only this CTA's shared memory, TMEM and the
-  // kernel parameters, so it may overlap the previous kernel in the stream;
-  // from here on global memory is read and written, after that kernel ends.
-  pdl_wait();
+  // Reads and writes. The kernel reads only its inputs (the pool, the batch
+  // descriptors, q, kq, vq), which no library kernel that releases its
+  // dependents early writes, so producers, MMA and softmax start while the
+  // previous kernel in the stream finishes; every thread that writes global
+  // memory (the impact zeroing, the item offsets, the epilogue) first waits
+  // for that kernel to complete (pdl_wait is free once it has).
 
   // zero the impact accumulator for the impact pass that follows
   if (p.impact_zero) {
+    pdl_wait();
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + tid; i < p.impact_len;
          i += int64_t(gridDim.x) * blockDim.x)
       p.impact_zero[i] = 0.f;
@@ -244,6 +247,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   if (blockIdx.x == 0 && p.item_prefix) {
+    pdl_wait();   // the previous call's combine may still read the offsets
     for (int b = tid; b <= B; b += blockDim.x) p.item_prefix[b] = prefix[b];
   }
 
@@ -426,6 +430,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         continue;
       }
+      pdl_wait();   // outputs and partials may still be read by the previous kernel
       float o[kHeadDim];
       if (n > 0) {
 #pragma unroll
@@ -820,44 +825,52 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p
   const int base = __ldcg(p.item_prefix + b);
   const size_t first = size_t(base) + size_t(g) * sh.n_split * sh.n_rt + rb;
   if (first + size_t(sh.n_split - 1) * sh.n_rt >= size_t(p.max_items)) return;
-  // statistics of every split first (lane s holds split s, 32 at a time), then
-  // the weighted rows with several loads in flight; split s weighs its own
-  // average O_s/l_s by l_s * 2^(m_s - m)
+  // Two round trips for up to 32 splits: lane s reads split s's (m, l) and
+  // turns it into the split's weight l_s 2^(m_s - m); then every split's
+  // fp16 row (4 columns per lane) is read at once and summed with the
+  // weights broadcast from their lanes. Split s holds its own average O_s/l_s.
   const float* row0 = p.part + (first * kFwdRows + rr) * kPartStride;
   const size_t split_stride = size_t(sh.n_rt) * kFwdRows * kPartStride;
   constexpr int kStatOff = kHeadDim / 2;   // 32-bit word of m (then l) in a row
+  // (m, l) of the first 32 splits stay in their lanes from the max pass
+  float2 ml0 = make_float2(-INFINITY, 0.f);
   float m = -INFINITY;
   for (int s0 = 0; s0 < sh.n_split; s0 += 32) {
     const int s = s0 + lane;
-    const float ms = s < sh.n_split ? __ldcg(row0 + s * split_stride + kStatOff) : -INFINITY;
-    float mm = ms;
+    const float2 mls = s < sh.n_split ? __ldcg(reinterpret_cast<const float2*>(row0 + s * split_stride + kStatOff))
+                                      : make_float2(-INFINITY, 0.f);
+    if (s0 == 0) ml0 = mls;
+    float mm = mls.x;
     for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
     m = fmaxf(m, mm);
   }
   const float m_use = (m == -INFINITY) ? 0.f : m;
   float l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < sh.n_split; s0 += 8) {
-    uint2 v[8];
-    float2 ml[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (s0 + j < sh.n_split) {
-        const float* row = row0 + (s0 + j) * split_stride;
-        ml[j] = __ldcg(reinterpret_cast<const float2*>(row + kStatOff));
-        v[j] = __ldcg(reinterpret_cast<const uint2*>(row) + lane);
-      } else {
-        ml[j] = make_float2(-INFINITY, 0.f);
-        v[j] = make_uint2(0u, 0u);
-      }
+  for (int s0 = 0; s0 < sh.n_split; s0 += 32) {
+    const int ns = min(32, sh.n_split - s0);
+    float wl = 0.f;
+    if (lane < ns) {
+      const float2 ml = s0 == 0 ? ml0
+                                : __ldcg(reinterpret_cast<const float2*>(row0 + (s0 + lane) * split_stride + kStatOff));
+      wl = (ml.x == -INFINITY) ? 0.f : ml.y * ex2(ml.x - m_use);
     }
+    float ws = wl;
+    for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
+    l += ws;
+    for (int j0 = 0; j0 < ns; j0 += 16) {
+      uint2 v[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float wgt = (ml[j].x == -INFINITY) ? 0.f : ml[j].y * ex2(ml[j].x - m_use);
-      const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&v[j].x));
-      const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&v[j].y));
-      l += wgt;
-      acc.x += lo.x * wgt; acc.y += lo.y * wgt; acc.z += hi.x * wgt; acc.w += hi.y * wgt;
+      for (int j = 0; j < 16; ++j)
+        v[j] = (j0 + j < ns) ? __ldcg(reinterpret_cast<const uint2*>(row0 + (s0 + j0 + j) * split_stride) + lane)
+                             : make_uint2(0u, 0u);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float wgt = __shfl_sync(0xffffffffu, wl, (j0 + j) & 31);
+        const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&v[j].x));
+        const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&v[j].y));
+        acc.x += lo.x * wgt; acc.y += lo.y * wgt; acc.z += hi.x * wgt; acc.w += hi.y * wgt;
+      }
     }
   }
   const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -880,7 +893,8 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p
 // theta_i = base^(-2 i / 128), as (cos, sin), computed in fp64 and stored in
 // fp32. One block per request.
 __global__ void __launch_bounds__(256) rope_table_kernel(const BatchDev B, double base, float2* table) {
-  pdl_launch_dependents();
+  // no early release: the attention kernel reads the table before its own
+  // wait, so it must start only once the table is complete
   const ReqInfo r = load_req(B, blockIdx.x);
   if (!req_ok(B, r)) return;
   pdl_wait();   // the kernel before this one may still read the table of the previous call

@@ -13,11 +13,13 @@
 //                   gathered through the page table (TMA page boxes)
 //   MMA warp      : S^T (128 keys x N rows) = K (smem) x Q^T (smem) -> TMEM,
 //                   two S buffers ahead of the epilogue
-//   8 epilogue warps: two per TMEM lane quarter, each over half of the rows;
-//                   per key 2^(s c + b_row), with the row's normaliser folded
-//                   into the bias b_row = log2(1 / (l H_q)) - m2, summed on
-//                   MUFU exp2 with packed fp32 pair arithmetic; each half
-//                   adds its column sum with one atomicAdd per key
+//   16 epilogue warps: four per TMEM lane quarter, each over a quarter of
+//                   the rows (more warps hide the TMEM and barrier latencies
+//                   behind the exp2 unit); per key 2^(s c + b_row), with the
+//                   row's normaliser folded into the bias
+//                   b_row = log2(1 / (l H_q)) - m2, summed on MUFU exp2 with
+//                   packed fp32 pair arithmetic; each warp adds its column
+//                   sum with one atomicAdd per key
 // The producer and MMA warps start while the kernels before this one finish
 // (programmatic dependent launch); the epilogue waits for their row
 // statistics.
@@ -37,7 +39,10 @@ constexpr int kITileBytes = kBN * kHeadDim * 2;     // K tile
 constexpr int kIHalf = kITileBytes / 2;
 constexpr int kIQHalf = kImpactRows * 128;          // 256 rows x 64 d (bf16) per d-half
 constexpr int kIQBytes = 2 * kIQHalf;
-constexpr int kImpThreads = 352;              // 8 epilogue + producer + MMA + RoPE warps
+constexpr int kImpEpiWarps = 16;             // four per TMEM lane quarter, each over a quarter of the rows
+constexpr int kImpEpiThreads = kImpEpiWarps * 32;
+constexpr int kWarpProducer = kImpEpiWarps, kWarpMma = kImpEpiWarps + 1, kWarpRope = kImpEpiWarps + 2;
+constexpr int kImpThreads = (kImpEpiWarps + 3) * 32;   // epilogue + producer + MMA + RoPE warps
 
 struct ImpDesc {
   int32_t kind;      // 0 doc tile, 1 query-key tile
@@ -95,7 +100,7 @@ __device__ __forceinline__ ImpItem decode_imp_item(const ImpactParams& p, const 
   it.t_begin = min(it.split * p.tiles_per_split, n_tiles);
   it.t_end = min(it.t_begin + p.tiles_per_split, n_tiles);
   it.nrows = min(kImpactRows, it.req.n_q * G - it.rb * kImpactRows);
-  it.N = (it.nrows + 63) & ~63;   // two halves of whole 32-column TMEM loads
+  it.N = (it.nrows + 127) & ~127;   // four quarters of whole 32-column TMEM loads
   return it;
 }
 
@@ -113,7 +118,7 @@ __device__ __forceinline__ void imp_abort(ImpCtrl* c, int32_t* err) {
   }
 }
 
-__global__ void __launch_bounds__(kImpThreads, 1)
+__global__ void __maxnreg__(104)
 impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_kq, const ImpactParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -136,17 +141,19 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_init(&ctl->kempty[s], 1);
       mbar_init(&ctl->kconv[s], 1);
     }
-    for (int s = 0; s < 2; ++s) { mbar_init(&ctl->s_full[s], 1); mbar_init(&ctl->s_free[s], 256); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&ctl->s_full[s], 1); mbar_init(&ctl->s_free[s], kImpEpiThreads); }
     mbar_init(&ctl->teardown, 1);
-    for (int s = 0; s < kIDescSlots; ++s) { mbar_init(&ctl->desc_full[s], 1); mbar_init(&ctl->desc_empty[s], 8); }
+    for (int s = 0; s < kIDescSlots; ++s) { mbar_init(&ctl->desc_full[s], 1); mbar_init(&ctl->desc_empty[s], kImpEpiWarps); }
     ctl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tmem_alloc(&ctl->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) { tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_kq); }
+  if (warp == kWarpProducer && lane == 0) {
+    tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_kq);
+  }
   if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < B; base += 32) {
@@ -176,11 +183,12 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const uint32_t tmem = ctl->tmem_base;
   volatile int* abort_flag = &ctl->abort;
 
-  if (warp < 8) {
+  if (warp < kImpEpiWarps) {
     // ------------------------------------------------------------ epilogue: thread = key
-    // Two warps per TMEM lane quarter: warp w and w + 4 share 32 keys and take
-    // one half of the block's rows each; the halves meet in shared memory.
-    const int half = warp >> 2;
+    // Four warps per TMEM lane quarter: warps w, w + 4, w + 8, w + 12 share 32
+    // keys and take one quarter of the block's rows each; every warp adds its
+    // own column sums.
+    const int part = warp >> 2;
     const int k = (warp & 3) * 32 + lane;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     uint32_t t_glob = 0;
@@ -193,9 +201,9 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const ImpItem it = decode_imp_item(p, prefix, w);
       const int n = it.t_end - it.t_begin;
       if (n == 0) continue;
-      named_bar_sync(1, 256);
-      {
-        const int r = tid;   // 256 epilogue threads, one row each
+      named_bar_sync(1, kImpEpiThreads);
+      if (tid < kImpactRows) {
+        const int r = tid;   // one row each
         // per row: -m + log2(1 / (l * H_q)), so that 2^(s*c + bias) is the
         // row's normalised weight already divided by H_q (-inf: no row)
         float bias = -INFINITY;
@@ -207,10 +215,10 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         ctl->neg_m2[r] = bias;
       }
-      named_bar_sync(1, 256);
+      named_bar_sync(1, kImpEpiThreads);
       float* seg = p.impact + (it.req.doc0 + it.req.q0);
-      const int cols = it.N >> 1;         // rows of this half (multiple of 16)
-      const int c0 = half * cols;
+      const int cols = it.N >> 2;         // rows of this quarter (32 or 64)
+      const int c0 = part * cols;
       for (int i = 0; i < n; ++i) {
         const uint32_t t = t_glob + i;
         const uint32_t buf = t & 1;
@@ -291,7 +299,7 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         tc_fence_before();
         mbar_arrive(&ctl->s_free[buf]);
-        // each half adds its own column sum: no barrier between the halves
+        // each quarter adds its own column sum: no barrier between them
         const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
         const float total = (a01.x + a01.y) + (a23.x + a23.y);
         if (valid) atomicAdd(seg + lpos, total);
@@ -299,7 +307,7 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       t_glob += n;
     }
     if (bad) imp_abort(ctl, p.err);
-  } else if (warp == 8) {
+  } else if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
     uint32_t t_glob = 0, q_iter = 0;
     int bad = 0;
@@ -383,7 +391,7 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (q_iter > 0) mbar_wait(&ctl->q_full, (q_iter - 1) & 1, &zero);
     }
     __syncwarp();
-  } else if (warp == 10) {
+  } else if (warp == kWarpRope) {
     // ------------------------------------------------------------ RoPE re-basing of the K tiles
     if (p.rope) {
       uint32_t t_glob = 0;
@@ -406,7 +414,7 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       __syncwarp();
     }
   } else {
-    // ------------------------------------------------------------ MMA issuer (warp 9)
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t q_base = smem_u32(sQ);
       uint32_t t_glob = 0, q_iter = 0;
@@ -450,7 +458,7 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

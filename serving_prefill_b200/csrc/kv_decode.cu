@@ -11,8 +11,8 @@
 // t % 16 of page page_ids[t / 16]; slots past the chunk's end are zeroed.
 //
 // One CTA per page of the batch: 16 slots x H_kv heads x 128 channels for K
-// and for V; a thread makes 8 channels (one 16-byte store) at a time. The
-// work is a stream from codes to pages, bound by HBM.
+// and for V; a thread makes 8 channels of one head (16-byte stores) for all 16
+// slots. The work is a stream from codes to pages, bound by HBM.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -23,7 +23,8 @@ namespace rag {
 constexpr int kDecThreads = 256;
 
 __global__ void __launch_bounds__(kDecThreads) kv_decode_kernel(const KvDecodeParams p) {
-  pdl_launch_dependents();
+  // no early release: the attention kernel reads pool pages before its own
+  // wait, so it must start only once every page written here is complete
   const int gp = blockIdx.x;   // page of the batch
   // chunk of this page: last c with chunk_page_off[c] <= gp
   int lo = 0, hi = p.n_chunks - 1;
@@ -47,42 +48,54 @@ __global__ void __launch_bounds__(kDecThreads) kv_decode_kernel(const KvDecodePa
   }
   const int hk = p.num_kv_heads;
   const int code_row = kHeadDim * p.bits / 8;                  // bytes of one token and head
-  const int units = 2 * kPage * hk * (kHeadDim / 8);            // 8-channel groups, K and V
   const int64_t page_base = (int64_t(p.layer) * p.num_pages + page) * hk * kPage * kHeadDim;
-  for (int u = threadIdx.x; u < units; u += kDecThreads) {
-    const int tensor = u / (units / 2);
-    const int r = u % (units / 2);
-    const int grp = r % (kHeadDim / 8);                         // channels 8 grp .. 8 grp + 7
-    const int h = (r / (kHeadDim / 8)) % hk;
-    const int slot = r / (kHeadDim / 8) / hk;
-    const int t = (gp - pg0) * kPage + slot;                    // token of the chunk
-    uint4 out = make_uint4(0u, 0u, 0u, 0u);
-    if (t < n_tok) {
-      const uint8_t* codes = (tensor ? p.codes_v : p.codes_k) + (int64_t(t0 + t) * hk + h) * code_row;
-      uint32_t q[8];
-      if (p.bits == 8) {
-        const uint2 w = __ldg(reinterpret_cast<const uint2*>(codes + grp * 8));
+  const int n_valid = min(kPage, n_tok - (gp - pg0) * kPage);   // slots of this page holding tokens
+  const int t_first = t0 + (gp - pg0) * kPage;
+  // A thread owns one (tensor, KV head, 8-channel group): its scale and offset
+  // are loaded once, then the codes of all 16 slots are loaded before the
+  // first value is computed (16 loads in flight), and 16 stores follow.
+  for (int u = threadIdx.x; u < 2 * hk * (kHeadDim / 8); u += kDecThreads) {
+    const int tensor = u / (hk * (kHeadDim / 8));
+    const int h = (u / (kHeadDim / 8)) % hk;
+    const int grp = u % (kHeadDim / 8);                        // channels 8 grp .. 8 grp + 7
+    const int64_t so = (int64_t(c) * hk + h) * kHeadDim + grp * 8;
+    const float4* scale = reinterpret_cast<const float4*>((tensor ? p.scale_v : p.scale_k) + so);
+    const float4* offset = reinterpret_cast<const float4*>((tensor ? p.offset_v : p.offset_k) + so);
+    const float4 s0 = __ldg(scale), s1 = __ldg(scale + 1), o0 = __ldg(offset), o1 = __ldg(offset + 1);
+    const uint8_t* codes = (tensor ? p.codes_v : p.codes_k) + (int64_t(t_first) * hk + h) * code_row;
+    const int64_t token_stride = int64_t(hk) * code_row;
+    uint2 cw[kPage];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) { q[j] = (w.x >> (8 * j)) & 0xffu; q[4 + j] = (w.y >> (8 * j)) & 0xffu; }
-      } else {
-        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(codes + grp * 4));
-#pragma unroll
-        for (int j = 0; j < 8; ++j) q[j] = (w >> (4 * j)) & 0xfu;
-      }
-      const int64_t sc = (int64_t(c) * hk + h) * kHeadDim + grp * 8;
-      const float* scale = (tensor ? p.scale_v : p.scale_k) + sc;
-      const float* offset = (tensor ? p.offset_v : p.offset_k) + sc;
-      const float4 s0 = __ldg(reinterpret_cast<const float4*>(scale));
-      const float4 s1 = __ldg(reinterpret_cast<const float4*>(scale) + 1);
-      const float4 o0 = __ldg(reinterpret_cast<const float4*>(offset));
-      const float4 o1 = __ldg(reinterpret_cast<const float4*>(offset) + 1);
-      out.x = pack_bf16x2(__fmaf_rn(float(q[0]), s0.x, o0.x), __fmaf_rn(float(q[1]), s0.y, o0.y));
-      out.y = pack_bf16x2(__fmaf_rn(float(q[2]), s0.z, o0.z), __fmaf_rn(float(q[3]), s0.w, o0.w));
-      out.z = pack_bf16x2(__fmaf_rn(float(q[4]), s1.x, o1.x), __fmaf_rn(float(q[5]), s1.y, o1.y));
-      out.w = pack_bf16x2(__fmaf_rn(float(q[6]), s1.z, o1.z), __fmaf_rn(float(q[7]), s1.w, o1.w));
+    for (int slot = 0; slot < kPage; ++slot) {
+      cw[slot] = make_uint2(0u, 0u);
+      if (slot >= n_valid) continue;
+      const uint8_t* cs = codes + slot * token_stride;
+      if (p.bits == 8) cw[slot] = __ldg(reinterpret_cast<const uint2*>(cs + grp * 8));
+      else cw[slot].x = __ldg(reinterpret_cast<const uint32_t*>(cs + grp * 4));
     }
-    __nv_bfloat16* pool = tensor ? p.pool_v : p.pool_k;
-    reinterpret_cast<uint4*>(pool + page_base + (int64_t(h) * kPage + slot) * kHeadDim)[grp] = out;
+    uint4* out = reinterpret_cast<uint4*>((tensor ? p.pool_v : p.pool_k) + page_base) + h * kPage * (kHeadDim / 8) + grp;
+#pragma unroll
+    for (int slot = 0; slot < kPage; ++slot) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);   // slots past the chunk's end are zeroed
+      if (slot < n_valid) {
+        float q[8];
+        if (p.bits == 8) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            q[i] = float((cw[slot].x >> (8 * i)) & 0xffu);
+            q[4 + i] = float((cw[slot].y >> (8 * i)) & 0xffu);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) q[i] = float((cw[slot].x >> (4 * i)) & 0xfu);
+        }
+        v.x = pack_bf16x2(__fmaf_rn(q[0], s0.x, o0.x), __fmaf_rn(q[1], s0.y, o0.y));
+        v.y = pack_bf16x2(__fmaf_rn(q[2], s0.z, o0.z), __fmaf_rn(q[3], s0.w, o0.w));
+        v.z = pack_bf16x2(__fmaf_rn(q[4], s1.x, o1.x), __fmaf_rn(q[5], s1.y, o1.y));
+        v.w = pack_bf16x2(__fmaf_rn(q[6], s1.z, o1.z), __fmaf_rn(q[7], s1.w, o1.w));
+      }
+      out[slot * (kHeadDim / 8)] = v;
+    }
   }
 }
 

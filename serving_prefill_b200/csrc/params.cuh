@@ -168,7 +168,7 @@ __host__ __device__ inline RcPlanLayout rc_plan_layout(int64_t max_tok, int64_t 
   l.words = at;
   return l;
 }
-enum : int32_t { kRcHdrTok = 0, kRcHdrCow = 1, kRcHdrNeeded = 2, kRcHdrErr = 3 };
+enum : int32_t { kRcHdrTok = 0, kRcHdrCow = 1, kRcHdrNeeded = 2, kRcHdrErr = 3, kRcHdrBySel = 4 };
 enum : int32_t { kRcErrNoFree = 16 };   // error bit beyond the device error bits: too few free pages
 
 struct RcPlanParams {
@@ -217,8 +217,8 @@ cudaError_t launch_kv_decode(const KvDecodeParams&, int total_pages, cudaStream_
 
 cudaError_t launch_rc_plan(const RcPlanParams&, cudaStream_t);
 cudaError_t launch_rc_copy(const RcCopyParams&, int grid, cudaStream_t);
-cudaError_t launch_rc_gemm(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const RcGemmParams&, int grid,
-                           cudaStream_t);
+cudaError_t launch_rc_gemm(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                           const RcGemmParams&, int grid, cudaStream_t);
 
 cudaError_t launch_attn_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                             const CUtensorMap&, const FwdParams&, int, cudaStream_t);

@@ -22,6 +22,8 @@
 //                     rounds each row to bf16 and stores it into its slot of
 //                     its private page (one KV head per output tile).
 // Every wait is bounded; a timeout raises a device error instead of hanging.
+// None of these kernels releases its dependents early: they write page tables
+// and pool pages, which the attention kernel reads before its own wait.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -76,7 +78,6 @@ __global__ void __launch_bounds__(kRcPlanThreads, 1) rc_plan_kernel(const RcPlan
   int32_t* cow_dst = p.plan + p.lay.cow_dst;
   int32_t* cow_mask = p.plan + p.lay.cow_mask;
   uint32_t* flags = reinterpret_cast<uint32_t*>(p.plan + p.lay.flags);
-  pdl_launch_dependents();
   if (tid == 0) s_err = 0;
   pdl_wait();   // the selection comes from the kernel before this one
 
@@ -183,18 +184,18 @@ __global__ void __launch_bounds__(kRcPlanThreads, 1) rc_plan_kernel(const RcPlan
     hdr[kRcHdrCow] = fits ? n_needed : 0;
     hdr[kRcHdrNeeded] = n_needed;
     hdr[kRcHdrErr] = s_err | (fits ? 0 : kRcErrNoFree);
+    hdr[kRcHdrBySel] = p.by_selection;   // rows t of the hidden states are consecutive
   }
 }
 
 // ---------------------------------------------------------------- copy
 
 constexpr int kRcCopyThreads = 256;
-constexpr int kRcCopyUnroll = 8;
+constexpr int kRcCopyUnroll = 16;
 
 // One private page per block iteration: K and V of this layer, every KV head,
-// every slot the selection does not overwrite (16-byte units, 8 in flight).
+// every slot the selection does not overwrite (16-byte units, 16 in flight).
 __global__ void __launch_bounds__(kRcCopyThreads) rc_copy_kernel(const RcCopyParams p) {
-  pdl_launch_dependents();
   pdl_wait();   // the plan comes from the kernel before this one
   const int32_t* hdr = p.plan;
   const int n_cow = __ldcg(hdr + kRcHdrCow);
@@ -265,13 +266,13 @@ __device__ __forceinline__ void rc_abort(RcCtrl* c, int32_t* err) {
 }
 
 __global__ void __launch_bounds__(kRcThreads, 1)
-rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wk,
-               const __grid_constant__ CUtensorMap tm_wv, const RcGemmParams p) {
+rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xt,
+               const __grid_constant__ CUtensorMap tm_wk, const __grid_constant__ CUtensorMap tm_wv,
+               const RcGemmParams p) {
   extern __shared__ uint8_t rc_smem_raw[];
   uint8_t* smem = rc_smem_raw + ((1024 - (smem_u32(rc_smem_raw) & 1023)) & 1023);
   RcCtrl* ctl = reinterpret_cast<RcCtrl*>(smem + kRcStages * kRcStageBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  pdl_launch_dependents();
   if (tid == 0) {
     for (int s = 0; s < kRcStages; ++s) { mbar_init(&ctl->full[s], 1); mbar_init(&ctl->empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&ctl->acc_full[b], 1); mbar_init(&ctl->acc_empty[b], 128); }
@@ -282,7 +283,9 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     tmem_alloc(&ctl->tmem_base, 256);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) { tma_prefetch_desc(&tm_x); tma_prefetch_desc(&tm_wk); tma_prefetch_desc(&tm_wv); }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_x); tma_prefetch_desc(&tm_xt); tma_prefetch_desc(&tm_wk); tma_prefetch_desc(&tm_wv);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -300,6 +303,10 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
+    // Hidden states listed by selection rank are consecutive rows: one tiled
+    // box of 128 rows per stage. Listed by doc position they are scattered:
+    // 32 gather4 loads of four rows each (one per lane).
+    const bool tiled = __ldcg(p.plan + kRcHdrBySel) != 0;
     uint32_t it = 0;
     int bad = 0;
     for (int tile = blockIdx.x; tile < n_tiles && !bad; tile += gridDim.x) {
@@ -323,7 +330,12 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         uint8_t* sa = smem + s * kRcStageBytes;
         if (lane == 0) mbar_arrive_expect_tx(&ctl->full[s], kRcStageBytes);
         __syncwarp();
-        tma_gather4(sa + lane * 4 * 128, &tm_x, &ctl->full[s], ks * kRcBK, r[0], r[1], r[2], r[3]);
+        if (tiled) {
+          // rows past x_rows are filled with zeros; the epilogue stores nothing for them
+          if (lane == 0) tma_load_2d(sa, &tm_xt, &ctl->full[s], ks * kRcBK, m0);
+        } else {
+          tma_gather4(sa + lane * 4 * 128, &tm_x, &ctl->full[s], ks * kRcBK, r[0], r[1], r[2], r[3]);
+        }
         if (lane == 0) tma_load_2d(sa + kRcABytes, tb, &ctl->full[s], ks * kRcBK, brow);
       }
     }
@@ -434,13 +446,13 @@ cudaError_t launch_rc_copy(const RcCopyParams& p, int grid, cudaStream_t stream)
   return launch_pdl(rc_copy_kernel, dim3(grid), dim3(kRcCopyThreads), 0, stream, 1, p);
 }
 
-cudaError_t launch_rc_gemm(const CUtensorMap& tx, const CUtensorMap& twk, const CUtensorMap& twv,
-                           const RcGemmParams& p, int grid, cudaStream_t stream) {
+cudaError_t launch_rc_gemm(const CUtensorMap& tx, const CUtensorMap& txt, const CUtensorMap& twk,
+                           const CUtensorMap& twv, const RcGemmParams& p, int grid, cudaStream_t stream) {
   const size_t smem = rc_gemm_smem_bytes();
   static SmemAttr attr;
   cudaError_t e = ensure_smem_attr(rc_gemm_kernel, attr, smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(rc_gemm_kernel, dim3(grid), dim3(kRcThreads), smem, stream, 1, tx, twk, twv, p);
+  return launch_pdl(rc_gemm_kernel, dim3(grid), dim3(kRcThreads), smem, stream, 1, tx, txt, twk, twv, p);
 }
 
 }  // namespace rag

@@ -318,6 +318,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   k = min(min(k, n), min(p.k_cap, p.k_max));
   int32_t* out_idx = p.topk_idx + int64_t(b) * p.k_cap;
   float* out_val = p.topk_val ? p.topk_val + int64_t(b) * p.k_cap : nullptr;
+  pdl_wait();   // the impact vector comes from the kernel before this one; outputs are written after it
   if (crank == 0) {
     if (p.k_out && tid == 0) p.k_out[b] = k;
     for (int i = k + tid; i < p.k_cap; i += kTopkThreads) {
@@ -326,7 +327,6 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     }
   }
   if (k == 0) return;   // the whole cluster leaves together
-  pdl_wait();           // the impact vector comes from the kernel before this one
 
   // Pass 1: histogram of the 12-bit buckets (sign, exponent, 3 mantissa bits)
   // of this CTA's slice, then the request's histogram and, per bucket, how

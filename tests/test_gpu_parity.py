@@ -169,3 +169,34 @@ def test_parity_full_size_32_layers():
     torch.cuda.synchronize()
     check_layer(case, 0, with_impact=False)
     check_layer(case, w.num_layers - 1, with_impact=True)
+
+
+def test_host_step_matches_the_device_step():
+    """The pipelined step from pinned host buffers (copies on their own
+    streams, ordered by events) gives the same outputs as the plain step,
+    twice in a row."""
+    from serving_prefill_b200.engine import HostStep
+    w = CASES["gqa4_rows3"]
+    case = DeviceCase(w)
+    layers = [(l,) + case.dev_inputs[l] for l in case.layers]
+    outs = [torch.empty_like(case.engine.o) for _ in layers]
+    case.engine.step(layers, w.impact_layer_index, outs=outs)
+    torch.cuda.synchronize()
+    want_o = [o.clone() for o in outs]
+    want_idx = case.engine.topk_idx.clone()
+    host_in = [tuple(t.cpu().pin_memory() for t in case.dev_inputs[l]) for l in case.layers]
+    dev_in = [(l,) + tuple(torch.empty_like(t) for t in case.dev_inputs[l]) for l in case.layers]
+    dev_out = [torch.empty_like(o) for o in outs]
+    host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+    host_topk = torch.empty_like(want_idx, device="cpu").pin_memory()
+    desc = [t.contiguous().pin_memory() for t in case.batch.host]
+    step = HostStep(case.engine, dev_in, dev_out, host_in, host_out, w.impact_layer_index, host_topk=host_topk,
+                    batch_host=desc)
+    for _ in range(2):
+        step()
+        torch.cuda.synchronize()
+        for a, b in zip(host_out, want_o):
+            assert torch.equal(a[: case.batch.total_q], b[: case.batch.total_q].cpu())   # O is run-to-run stable
+        # the selection that came back is the one on the device (Impact sums by
+        # atomics, so near-ties may order differently from the first run)
+        assert torch.equal(host_topk, case.engine.topk_idx.cpu())
