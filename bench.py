@@ -411,7 +411,7 @@ def recompute_work(w, n_tok, n_cow):
     return {"gemm_flops": gemm_flops, "gemm_bytes": gemm_bytes, "copy_bytes": copy_bytes}
 
 
-def run_recompute(args, w, device, do_cpu):
+def run_recompute(args, w, device, do_cpu, ncu=False):
     """Plan once, then every layer's page copy and K/V projection for the
     selection the fused step made on the workload's selecting layer."""
     import serving_prefill_b200 as sp
@@ -451,6 +451,11 @@ def run_recompute(args, w, device, do_cpu):
     st, counts = sp.rag_recompute_status(plan)
     if st != 0:
         raise RuntimeError(f"recompute status {st}")
+    if ncu:   # profiling mode: eager steps only
+        for _ in range(args.warmup + args.steps):
+            step()
+        torch.cuda.synchronize()
+        return sp.rag_recompute_status(plan)[0]
     n_tok, n_cow, _ = counts
     s_cap = torch.cuda.Stream()
     s_cap.wait_stream(torch.cuda.current_stream())
@@ -592,7 +597,7 @@ def decode_bits(w, layer):
     return 8 if layer < w.num_layers // 2 else 4
 
 
-def run_kv_decode(args, w, device, do_cpu):
+def run_kv_decode(args, w, device, do_cpu, ncu=False):
     """Every layer of every distinct chunk decoded from its quantized stream into the pool."""
     import serving_prefill_b200 as sp
     from serving_prefill_b200 import KVPool
@@ -618,6 +623,11 @@ def run_kv_decode(args, w, device, do_cpu):
     torch.cuda.synchronize()
     if int(err.item()) != 0:
         raise RuntimeError(f"kv decode device error {int(err.item())}")
+    if ncu:   # profiling mode: eager steps only
+        for _ in range(args.warmup + args.steps):
+            step(dev)
+        torch.cuda.synchronize()
+        return int(err.item())
     s_cap = torch.cuda.Stream()
     s_cap.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()
@@ -884,6 +894,8 @@ def main():
                     help="measure the headline workload only (no per_config block)")
     ap.add_argument("--ncu", action="store_true",
                     help="profiling mode: one input copy, eager launches, W + K steps, no JSON")
+    ap.add_argument("--ncu-path", default="step", choices=["step", "recompute", "kv_decode"],
+                    help="with --ncu: the fused step, the selective recompute or the KV decode")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     w = get_workload(args.config)
@@ -915,6 +927,11 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     device = local
+    if args.ncu and args.ncu_path != "step":
+        run = run_recompute if args.ncu_path == "recompute" else run_kv_decode
+        st = run(args, w, device, False, ncu=True)
+        print(f"ncu mode: {args.warmup + args.steps} eager steps of {args.ncu_path} on {w.name}, status {st}")
+        sys.exit(0 if st == 0 else 1)
     if args.ncu:
         torch.cuda.set_device(device)
         lay = make_layout(w)

@@ -366,6 +366,10 @@ RAG_API rag_status rag_last_device_error(void* workspace, int32_t* bits, void* s
  * RAG_ERR_TIMEOUT. */
 RAG_API rag_status rag_selftest_wait_timeout(int32_t* device_err, int64_t limit_ns, void* stream);
 
+/* Name of the last CUDA runtime error a call of this library met (the detail
+ * behind a RAG_ERR_CUDA return), or "cudaSuccess". Host function. */
+RAG_API const char* rag_last_cuda_error(void);
+
 /* Kernel launches this library has made in this process (all entry points). */
 RAG_API int64_t rag_launch_count(void);
 

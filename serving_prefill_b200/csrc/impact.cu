@@ -118,7 +118,9 @@ __device__ __forceinline__ void imp_abort(ImpCtrl* c, int32_t* err) {
   }
 }
 
-__global__ void __maxnreg__(104)
+// 19 warps: one SM sub-partition holds five of them, so the register count is
+// bounded by 16,384 / (5 * 32) (ptxas derives it from the launch bounds)
+__global__ void __launch_bounds__(kImpThreads, 1)
 impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_kq, const ImpactParams p) {
   extern __shared__ uint8_t smem_raw[];

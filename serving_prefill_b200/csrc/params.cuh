@@ -63,6 +63,24 @@ inline cudaError_t ensure_smem_attr(Kernel kernel, SmemAttr& rec, size_t bytes) 
   return cudaSuccess;
 }
 
+// The last CUDA error a library call met (reported by rag_last_cuda_error).
+void note_cuda_error(cudaError_t e);
+
+// Ordinary launch (waits for the previous kernel to complete) that returns
+// this launch's own error rather than a stale one from an earlier call.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_plain(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 struct FwdParams {
   BatchDev batch;
   int32_t num_pages, num_kv_heads, num_q_heads, group, layer;

@@ -44,8 +44,7 @@ __global__ void __launch_bounds__(256) pool_write_kernel(const PoolWriteParams p
 }
 
 cudaError_t launch_pool_write(const PoolWriteParams& p, int n_pages, cudaStream_t stream) {
-  pool_write_kernel<<<dim3(n_pages, p.num_kv_heads), 256, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_plain(pool_write_kernel, dim3(n_pages, p.num_kv_heads), dim3(256), 0, stream, p);
 }
 
 }  // namespace rag

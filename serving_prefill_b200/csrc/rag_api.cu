@@ -32,6 +32,11 @@ struct ProfRecord {
 };
 
 static std::atomic<int64_t> g_launches{0};
+static std::atomic<int> g_last_cuda_error{0};
+
+void note_cuda_error(cudaError_t e) {
+  if (e != cudaSuccess) g_last_cuda_error.store(int(e));
+}
 static std::atomic<int> g_prof_on{0};
 static std::mutex g_prof_mu;
 static std::vector<ProfRecord> g_prof;
@@ -72,6 +77,7 @@ struct LaunchScope {
   }
   void done(cudaError_t e) {
     if (e == cudaSuccess) g_launches.fetch_add(1);
+    else note_cuda_error(e);
     if (start) {
       record_event(stop, stream);
       std::lock_guard<std::mutex> lk(g_prof_mu);
@@ -656,7 +662,9 @@ rag_status rag_recompute_kv(const rag_kv_pool* pool, int32_t layer, const rag_ba
     cp.layer = layer;
     cp.num_pages = pool->num_pages;
     cp.num_kv_heads = H_kv;
-    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(int64_t(4) * sms, b.num_page_refs)));
+    // one CTA per SM: every CTA starts at once, so the projection is released
+    // as soon as the plan is visible and runs beside the copy
+    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(sms, b.num_page_refs)));
     LaunchScope ls(kKindRcCopy, s);
     cudaError_t e = launch_rc_copy(cp, grid, s);
     ls.done(e);
@@ -717,6 +725,10 @@ rag_status rag_last_device_error(void* workspace, int32_t* bits, void* stream) {
 }
 
 int64_t rag_launch_count(void) { return g_launches.load(); }
+
+const char* rag_last_cuda_error(void) {
+  return cudaGetErrorName(static_cast<cudaError_t>(g_last_cuda_error.load()));
+}
 
 void rag_profile_enable(int32_t on) { g_prof_on.store(on ? 1 : 0); }
 

@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(64, 1) wait_selftest_kernel(int32_t* err, uint
 extern "C" RAG_API rag_status rag_selftest_wait_timeout(int32_t* device_err, int64_t limit_ns, void* stream) {
   if (!device_err || limit_ns <= 0 || limit_ns > int64_t(rag::kWaitLimitNs)) return RAG_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  rag::wait_selftest_kernel<<<1, 64, 0, s>>>(device_err, uint64_t(limit_ns));
-  return cudaGetLastError() == cudaSuccess ? RAG_OK : RAG_ERR_CUDA;
+  const cudaError_t e = rag::launch_plain(rag::wait_selftest_kernel, dim3(1), dim3(64), 0, s, device_err,
+                                          uint64_t(limit_ns));
+  rag::note_cuda_error(e);
+  return e == cudaSuccess ? RAG_OK : RAG_ERR_CUDA;
 }

@@ -165,13 +165,12 @@ cudaError_t launch_simt_attn(const SimtParams& p, int total_q, cudaStream_t stre
   static SmemAttr attr;
   cudaError_t e = ensure_smem_attr(simt_attn_kernel, attr, smem);
   if (e != cudaSuccess) return e;
-  simt_attn_kernel<<<dim3(total_q, p.num_q_heads), kSimtThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_plain(simt_attn_kernel, dim3(total_q, p.num_q_heads), dim3(kSimtThreads), smem, stream, p);
 }
 
 cudaError_t launch_simt_impact(const SimtParams& p, int max_keys, int num_requests, cudaStream_t stream) {
-  simt_impact_kernel<<<dim3(max_keys, num_requests), kSimtThreads, sizeof(float) * p.head_dim, stream>>>(p);
-  return cudaGetLastError();
+  return launch_plain(simt_impact_kernel, dim3(max_keys, num_requests), dim3(kSimtThreads), sizeof(float) * p.head_dim,
+                      stream, p);
 }
 
 }  // namespace rag

@@ -32,7 +32,10 @@ STATUS = {
 
 class RagError(RuntimeError):
     def __init__(self, status: int, where: str):
-        super().__init__(f"{where}: {STATUS.get(status, 'unknown')} (status {status})")
+        detail = ""
+        if status == 5 and _lib is not None:
+            detail = f", {_lib.rag_last_cuda_error().decode()}"
+        super().__init__(f"{where}: {STATUS.get(status, 'unknown')} (status {status}{detail})")
         self.status = status
 
 
@@ -81,6 +84,7 @@ EXPORTS = {
                                    c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]),
     "rag_recompute_status": (c_int32, [c_void_p, c_void_p, c_void_p]),
     "rag_launch_count": (c_int64, []),
+    "rag_last_cuda_error": (ctypes.c_char_p, []),
     "rag_profile_enable": (None, [c_int32]),
     "rag_profile_collect": (c_int32, [c_void_p, c_void_p, c_int32]),
     "rag_profile_peek": (c_int32, [c_void_p, c_void_p, c_int32]),

@@ -120,3 +120,9 @@ def test_bucket_above_the_kth_longer_than_a_register_sort():
     seg = np.concatenate([low[:40000], a, low[40000:], b])
     n = len(seg)
     check([seg], 12000.5 / n)                  # k = 12,000: all of a, 2,000 of b
+
+
+def test_whole_sort_boundary():
+    # 4,096 doc tokens are sorted whole by one CTA; 4,097 take the bucket path
+    rng = np.random.default_rng(12)
+    check([rng.random(4096), rng.lognormal(-4, 1.0, 4097), rng.integers(0, 3, 4096).astype(np.float64)], 0.15)
