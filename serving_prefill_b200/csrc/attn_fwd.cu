@@ -102,7 +102,7 @@ __device__ __forceinline__ FwdItem decode_fwd_item(const FwdParams& p, const int
   it.split = local % sh.n_split;
   it.g = local / sh.n_split;
   const int rows = it.req.n_q * p.group - it.rb * kFwdRows;
-  it.n_qt = rows > kBM ? 2 : 1;
+  it.n_qt = (rows > kBM && kFwdRows > kBM) ? 2 : 1;   // Q tiles holding rows of this block
   it.n_doc_tiles = doc_tiles(it.req);
   const int last_tok = min(it.req.n_q, (it.rb + 1) * kFwdRows / p.group) - 1;
   const int n_tiles = it.n_doc_tiles + query_tiles_upto(last_tok);
@@ -470,7 +470,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // partial row: this split's own softmax average O/l in fp16 (|O/l| is
         // bounded by max |V|), then its reference max m and sum l in fp32
         const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(p.part + ((size_t(w) * kQTiles + qt) * kBM + r) * kPartStride);
+        uint4* dst = reinterpret_cast<uint4*>(p.part + (size_t(w) * kFwdRows + qt * kBM + r) * kPartStride);
 #pragma unroll
         for (int c = 0; c < kHeadDim / 8; ++c) {
           uint4 v;
@@ -825,52 +825,44 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p
   const int base = __ldcg(p.item_prefix + b);
   const size_t first = size_t(base) + size_t(g) * sh.n_split * sh.n_rt + rb;
   if (first + size_t(sh.n_split - 1) * sh.n_rt >= size_t(p.max_items)) return;
-  // Two round trips for up to 32 splits: lane s reads split s's (m, l) and
-  // turns it into the split's weight l_s 2^(m_s - m); then every split's
-  // fp16 row (4 columns per lane) is read at once and summed with the
-  // weights broadcast from their lanes. Split s holds its own average O_s/l_s.
+  // statistics of every split first (lane s holds split s, 32 at a time), then
+  // the weighted rows with several loads in flight; split s weighs its own
+  // average O_s/l_s by l_s * 2^(m_s - m)
   const float* row0 = p.part + (first * kFwdRows + rr) * kPartStride;
   const size_t split_stride = size_t(sh.n_rt) * kFwdRows * kPartStride;
   constexpr int kStatOff = kHeadDim / 2;   // 32-bit word of m (then l) in a row
-  // (m, l) of the first 32 splits stay in their lanes from the max pass
-  float2 ml0 = make_float2(-INFINITY, 0.f);
   float m = -INFINITY;
   for (int s0 = 0; s0 < sh.n_split; s0 += 32) {
     const int s = s0 + lane;
-    const float2 mls = s < sh.n_split ? __ldcg(reinterpret_cast<const float2*>(row0 + s * split_stride + kStatOff))
-                                      : make_float2(-INFINITY, 0.f);
-    if (s0 == 0) ml0 = mls;
-    float mm = mls.x;
+    const float ms = s < sh.n_split ? __ldcg(row0 + s * split_stride + kStatOff) : -INFINITY;
+    float mm = ms;
     for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
     m = fmaxf(m, mm);
   }
   const float m_use = (m == -INFINITY) ? 0.f : m;
   float l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < sh.n_split; s0 += 32) {
-    const int ns = min(32, sh.n_split - s0);
-    float wl = 0.f;
-    if (lane < ns) {
-      const float2 ml = s0 == 0 ? ml0
-                                : __ldcg(reinterpret_cast<const float2*>(row0 + (s0 + lane) * split_stride + kStatOff));
-      wl = (ml.x == -INFINITY) ? 0.f : ml.y * ex2(ml.x - m_use);
-    }
-    float ws = wl;
-    for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
-    l += ws;
-    for (int j0 = 0; j0 < ns; j0 += 16) {
-      uint2 v[16];
+  for (int s0 = 0; s0 < sh.n_split; s0 += 8) {
+    uint2 v[8];
+    float2 ml[8];
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
-        v[j] = (j0 + j < ns) ? __ldcg(reinterpret_cast<const uint2*>(row0 + (s0 + j0 + j) * split_stride) + lane)
-                             : make_uint2(0u, 0u);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float wgt = __shfl_sync(0xffffffffu, wl, (j0 + j) & 31);
-        const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&v[j].x));
-        const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&v[j].y));
-        acc.x += lo.x * wgt; acc.y += lo.y * wgt; acc.z += hi.x * wgt; acc.w += hi.y * wgt;
+    for (int j = 0; j < 8; ++j) {
+      if (s0 + j < sh.n_split) {
+        const float* row = row0 + (s0 + j) * split_stride;
+        ml[j] = __ldcg(reinterpret_cast<const float2*>(row + kStatOff));
+        v[j] = __ldcg(reinterpret_cast<const uint2*>(row) + lane);
+      } else {
+        ml[j] = make_float2(-INFINITY, 0.f);
+        v[j] = make_uint2(0u, 0u);
       }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float wgt = (ml[j].x == -INFINITY) ? 0.f : ml[j].y * ex2(ml[j].x - m_use);
+      const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&v[j].x));
+      const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&v[j].y));
+      l += wgt;
+      acc.x += lo.x * wgt; acc.y += lo.y * wgt; acc.z += hi.x * wgt; acc.w += hi.y * wgt;
     }
   }
   const float inv = l > 0.f ? 1.f / l : 0.f;

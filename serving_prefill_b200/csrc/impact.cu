@@ -13,13 +13,12 @@
 //                   gathered through the page table (TMA page boxes)
 //   MMA warp      : S^T (128 keys x N rows) = K (smem) x Q^T (smem) -> TMEM,
 //                   two S buffers ahead of the epilogue
-//   16 epilogue warps: four per TMEM lane quarter, each over a quarter of
-//                   the rows (more warps hide the TMEM and barrier latencies
-//                   behind the exp2 unit); per key 2^(s c + b_row), with the
-//                   row's normaliser folded into the bias
-//                   b_row = log2(1 / (l H_q)) - m2, summed on MUFU exp2 with
-//                   packed fp32 pair arithmetic; each warp adds its column
-//                   sum with one atomicAdd per key
+//   8 epilogue warps: two per TMEM lane quarter, each over half of the rows;
+//                   per key 2^(s c + b_row), with the row's normaliser folded
+//                   into the bias b_row = log2(1 / (l H_q)) - m2, summed on
+//                   MUFU exp2 with packed fp32 pair arithmetic; each half
+//                   adds its column sum with one atomicAdd per key (16 warps,
+//                   four per quarter, measured slower)
 // The producer and MMA warps start while the kernels before this one finish
 // (programmatic dependent launch); the epilogue waits for their row
 // statistics.
@@ -39,7 +38,8 @@ constexpr int kITileBytes = kBN * kHeadDim * 2;     // K tile
 constexpr int kIHalf = kITileBytes / 2;
 constexpr int kIQHalf = kImpactRows * 128;          // 256 rows x 64 d (bf16) per d-half
 constexpr int kIQBytes = 2 * kIQHalf;
-constexpr int kImpEpiWarps = 16;             // four per TMEM lane quarter, each over a quarter of the rows
+constexpr int kImpEpiWarps = 8;              // two per TMEM lane quarter, each over half of the rows
+constexpr int kImpParts = kImpEpiWarps / 4;  // row parts per TMEM lane quarter
 constexpr int kImpEpiThreads = kImpEpiWarps * 32;
 constexpr int kWarpProducer = kImpEpiWarps, kWarpMma = kImpEpiWarps + 1, kWarpRope = kImpEpiWarps + 2;
 constexpr int kImpThreads = (kImpEpiWarps + 3) * 32;   // epilogue + producer + MMA + RoPE warps
@@ -100,7 +100,7 @@ __device__ __forceinline__ ImpItem decode_imp_item(const ImpactParams& p, const 
   it.t_begin = min(it.split * p.tiles_per_split, n_tiles);
   it.t_end = min(it.t_begin + p.tiles_per_split, n_tiles);
   it.nrows = min(kImpactRows, it.req.n_q * G - it.rb * kImpactRows);
-  it.N = (it.nrows + 127) & ~127;   // four quarters of whole 32-column TMEM loads
+  it.N = (it.nrows + 32 * kImpParts - 1) / (32 * kImpParts) * (32 * kImpParts);   // parts of whole 32-column loads
   return it;
 }
 
@@ -118,8 +118,8 @@ __device__ __forceinline__ void imp_abort(ImpCtrl* c, int32_t* err) {
   }
 }
 
-// 19 warps: one SM sub-partition holds five of them, so the register count is
-// bounded by 16,384 / (5 * 32) (ptxas derives it from the launch bounds)
+// The launch bounds let ptxas bound the registers by what one SM
+// sub-partition's 16,384-register file holds for its share of the warps.
 __global__ void __launch_bounds__(kImpThreads, 1)
 impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_kq, const ImpactParams p) {
@@ -187,9 +187,9 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   if (warp < kImpEpiWarps) {
     // ------------------------------------------------------------ epilogue: thread = key
-    // Four warps per TMEM lane quarter: warps w, w + 4, w + 8, w + 12 share 32
-    // keys and take one quarter of the block's rows each; every warp adds its
-    // own column sums.
+    // kImpParts warps per TMEM lane quarter: warps w, w + 4, ... share 32 keys
+    // and take one part of the block's rows each; every warp adds its own
+    // column sums (no barrier between the parts).
     const int part = warp >> 2;
     const int k = (warp & 3) * 32 + lane;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
@@ -219,7 +219,7 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       named_bar_sync(1, kImpEpiThreads);
       float* seg = p.impact + (it.req.doc0 + it.req.q0);
-      const int cols = it.N >> 2;         // rows of this quarter (32 or 64)
+      const int cols = it.N / kImpParts;   // rows of this part (a multiple of 32)
       const int c0 = part * cols;
       for (int i = 0; i < n; ++i) {
         const uint32_t t = t_glob + i;
@@ -301,7 +301,7 @@ impact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         tc_fence_before();
         mbar_arrive(&ctl->s_free[buf]);
-        // each quarter adds its own column sum: no barrier between them
+        // each part adds its own column sum: no barrier between them
         const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
         const float total = (a01.x + a01.y) + (a23.x + a23.y);
         if (valid) atomicAdd(seg + lpos, total);

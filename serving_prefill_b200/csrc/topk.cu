@@ -3,9 +3,8 @@
 // takes max(1, int(doc_token_count * ratio)) and torch.topk over the doc slice
 // of the impact vector).
 //
-// A request of at most 4,096 doc tokens is sorted whole by one CTA (a bitonic
-// network over composite keys). Longer ones: a cluster of C CTAs per request
-// (C grows with the longest request, up to 8). Each CTA histograms the top 12 bits of its slice of the fp32 impacts
+// A cluster of C CTAs per request (C grows with the longest request, up to
+// 8). Each CTA histograms the top 12 bits of its slice of the fp32 impacts
 // (impacts are >= 0, so their bit patterns order like the values); the
 // cluster's histograms, read over distributed shared memory, give the bucket
 // d1 holding the k-th largest value and every bucket's place in descending
@@ -36,7 +35,6 @@ static_assert(kTopkMaxK <= kTopkSortMax, "the k selected keys must fit the stagi
 constexpr int kTopkMaxCluster = 8;
 constexpr int kTopkSlice = 8192;     // doc tokens per CTA before the cluster grows
 constexpr int kRankMax = 256;        // longest bucket ordered by counting ranks (longer: sorted)
-constexpr int kTopkDirectMax = 4096; // requests up to this many doc tokens are sorted whole
 
 struct TopkSmem {
   uint64_t staged[kTopkSortMax];     // composite keys of the buckets this CTA orders, at their final bucket ranges
@@ -330,19 +328,6 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   }
   if (k == 0) return;   // the whole cluster leaves together
 
-  // Short requests: one sorting network over every composite key beats the
-  // two passes of bucket work (histograms, scans, staging) on latency.
-  if (csize == 1 && n <= kTopkDirectMax) {
-    for (int i = tid; i < n; i += kTopkThreads) S.staged[i] = composite(impact_key(__ldg(keys + i)), i);
-    __syncthreads();
-    block_sort_any(S.staged, n);
-    for (int i = tid; i < k; i += kTopkThreads) {
-      const uint64_t comp = S.staged[i];
-      out_idx[i] = int32_t(comp & 0xffffffffu);
-      if (out_val) out_val[i] = __uint_as_float(~uint32_t(comp >> 32));
-    }
-    return;
-  }
 
   // Pass 1: histogram of the 12-bit buckets (sign, exponent, 3 mantissa bits)
   // of this CTA's slice, then the request's histogram and, per bucket, how

@@ -139,3 +139,8 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(rag, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         rag.lib()
+
+
+def test_last_cuda_error_names_a_cuda_error():
+    name = lib().rag_last_cuda_error().decode()
+    assert name.startswith("cuda")
