@@ -662,9 +662,7 @@ rag_status rag_recompute_kv(const rag_kv_pool* pool, int32_t layer, const rag_ba
     cp.layer = layer;
     cp.num_pages = pool->num_pages;
     cp.num_kv_heads = H_kv;
-    // one CTA per SM: every CTA starts at once, so the projection is released
-    // as soon as the plan is visible and runs beside the copy
-    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(sms, b.num_page_refs)));
+    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(int64_t(4) * sms, b.num_page_refs)));
     LaunchScope ls(kKindRcCopy, s);
     cudaError_t e = launch_rc_copy(cp, grid, s);
     ls.done(e);

@@ -22,11 +22,10 @@
 //                     rounds each row to bf16 and stores it into its slot of
 //                     its private page (one KV head per output tile).
 // Every wait is bounded; a timeout raises a device error instead of hanging.
-// The plan and the projection do not release their dependents early: they
-// write page tables and pool pages, which the attention kernel reads before
-// its own wait. The copy releases the projection once the plan is visible,
-// so the two (one bound by HBM, one by the tensor cores) run side by side;
-// the projection waits for the copy before it exits.
+// None of these kernels releases its dependents early: they write page tables
+// and pool pages, which the attention kernel reads before its own wait. (Running
+// the copy beside the projection measured slower: the projection streams its
+// operands from L2 at a high rate and the copy competes for it.)
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -200,11 +199,6 @@ constexpr int kRcCopyUnroll = 16;
 // every slot the selection does not overwrite (16-byte units, 16 in flight).
 __global__ void __launch_bounds__(kRcCopyThreads) rc_copy_kernel(const RcCopyParams p) {
   pdl_wait();   // the plan comes from the kernel before this one
-  // The projection that follows writes only the selected slots, which this
-  // kernel never touches, and reads only the plan (complete now) and its
-  // inputs: it may start at once and run beside the copy. It waits for this
-  // kernel before it exits, so the kernel after it sees every page complete.
-  pdl_launch_dependents();
   const int32_t* hdr = p.plan;
   const int n_cow = __ldcg(hdr + kRcHdrCow);
   const int hk = p.num_kv_heads;
@@ -297,9 +291,7 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // No wait here: the page copy before this kernel released it only once the
-  // plan was complete, and the two write disjoint bytes. The plan is read
-  // through L2 (ld.global.cg and TMA).
+  pdl_wait();   // the plan and the page copies come from the kernels before this one
 
   int32_t* err = p.plan + kRcHdrErr;
   const int n_tok = __ldcg(p.plan + kRcHdrTok);
@@ -444,7 +436,6 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
-  pdl_wait();   // this grid completes only after the page copy: the kernel after it sees whole pages
 }
 
 // ---------------------------------------------------------------- launchers
