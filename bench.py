@@ -341,7 +341,7 @@ def run_gpu(args, w, rank, world, device):
     roof["kernel"] = dom
     roof["peak_source"] = peaks["source"]
     roof["avg_launch_us"] = avg_s * 1e6
-    roof["traffic"] = recorded_traffic(args.config, dom)
+    roof["traffic"] = recorded_traffic(w.name, dom)
     t_roof = max(work["step_flops"] / (tflops_peak * 1e12), work["step_bytes"] / (peaks["hbm_gbs"] * 1e9))
     step_roof = {"t_roof_us": t_roof * 1e6, "t_step_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step / 1e3)}
 
