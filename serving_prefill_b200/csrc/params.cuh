@@ -213,6 +213,7 @@ struct RcGemmParams {
   RcPlanLayout lay;
   int32_t layer, num_pages, num_kv_heads, d_model;
   int32_t x_rows;
+  int32_t heads_per_tile;          // output heads per tile: 2 when num_kv_heads is even, else 1
   int64_t max_tok;
 };
 

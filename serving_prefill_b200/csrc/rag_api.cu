@@ -639,6 +639,7 @@ rag_status rag_recompute_kv(const rag_kv_pool* pool, int32_t layer, const rag_ba
   const RcPlanLayout lay = rc_plan_layout(int64_t(b.num_requests) * k_cap, b.num_page_refs);
   const int64_t max_tok = int64_t(b.num_requests) * k_cap;
   if (max_tok == 0) return RAG_OK;
+  const int hpt = (H_kv % 2 == 0) ? 2 : 1;   // output heads per projection tile
   CUtensorMap tm_x, tm_xt, tm_wk, tm_wv;
   {
     const uint64_t dx[2] = {uint64_t(d_model), uint64_t(x_rows)};
@@ -646,7 +647,7 @@ rag_status rag_recompute_kv(const rag_kv_pool* pool, int32_t layer, const rag_ba
     const uint32_t bx[2] = {64u, 1u};       // gather4: one row per box
     const uint32_t bxt[2] = {64u, 128u};    // consecutive rows: one 128-row box
     const uint64_t dw[2] = {uint64_t(d_model), uint64_t(H_kv) * kHeadDim};
-    const uint32_t bw[2] = {64u, 128u};
+    const uint32_t bw[2] = {64u, uint32_t(128 * hpt)};   // the rows of hpt heads
     if (!make_map(&tm_x, x, 2, dx, sx, bx) || !make_map(&tm_xt, x, 2, dx, sx, bxt) ||
         !make_map(&tm_wk, w_k, 2, dw, sx, bw) || !make_map(&tm_wv, w_v, 2, dw, sx, bw))
       return RAG_ERR_CUDA;
@@ -678,8 +679,9 @@ rag_status rag_recompute_kv(const rag_kv_pool* pool, int32_t layer, const rag_ba
   gp.num_kv_heads = H_kv;
   gp.d_model = d_model;
   gp.x_rows = int32_t(x_rows);
+  gp.heads_per_tile = hpt;
   gp.max_tok = max_tok;
-  const int64_t tiles_bound = ((max_tok + 127) / 128) * 2 * H_kv;
+  const int64_t tiles_bound = ((max_tok + 127) / 128) * (2 * H_kv / hpt);
   const int grid = int(std::max<int64_t>(1, std::min<int64_t>(sms, tiles_bound)));
   LaunchScope ls(kKindRcGemm, s);
   cudaError_t e = launch_rc_gemm(tm_x, tm_xt, tm_wk, tm_wv, gp, grid, s);

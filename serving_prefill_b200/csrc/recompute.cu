@@ -15,12 +15,14 @@
 //                     all KV heads); the selected slots are left to the GEMM,
 //                     so the two never write the same bytes
 //   GEMM (tcgen05)  : [K | V] rows = X_sel W^T. The A operand (128 selected
-//                     tokens x 64 hidden features per stage) is gathered by
-//                     TMA tile::gather4 straight from the hidden-state rows,
-//                     the B operand (128 rows of W_K or W_V) by a tiled TMA
-//                     load; the accumulator lives in TMEM, and the epilogue
-//                     rounds each row to bf16 and stores it into its slot of
-//                     its private page (one KV head per output tile).
+//                     tokens x 64 hidden features per stage) is loaded as one
+//                     tiled TMA box when the hidden states are listed by
+//                     selection rank, or gathered by TMA tile::gather4 from
+//                     rows listed by doc position; the B operand (the rows of
+//                     two KV heads of W_K or W_V, one when H_kv is odd) by a
+//                     tiled TMA load; the accumulator lives in TMEM, and the
+//                     epilogue rounds each row to bf16 and stores it into its
+//                     slot of its private page.
 // Every wait is bounded; a timeout raises a device error instead of hanging.
 // None of these kernels releases its dependents early: they write page tables
 // and pool pages, which the attention kernel reads before its own wait. (Running
@@ -192,18 +194,22 @@ __global__ void __launch_bounds__(kRcPlanThreads, 1) rc_plan_kernel(const RcPlan
 
 // ---------------------------------------------------------------- copy
 
-constexpr int kRcCopyThreads = 256;
-constexpr int kRcCopyUnroll = 16;
+constexpr int kRcCopyThreads = 512;   // 16 warps: one per (tensor, KV head) block of a page, up to 8 heads
 
 // One private page per block iteration: K and V of this layer, every KV head,
-// every slot the selection does not overwrite (16-byte units, 16 in flight).
-__global__ void __launch_bounds__(kRcCopyThreads) rc_copy_kernel(const RcCopyParams p) {
+// every slot the selection does not overwrite. A warp copies one (tensor,
+// head) block of 16 slots x 256 bytes: each lane moves eight 16-byte units,
+// all eight loads in flight before the first store.
+__global__ void __launch_bounds__(kRcCopyThreads, 2) rc_copy_kernel(const RcCopyParams p) {
   pdl_wait();   // the plan comes from the kernel before this one
   const int32_t* hdr = p.plan;
   const int n_cow = __ldcg(hdr + kRcHdrCow);
   const int hk = p.num_kv_heads;
-  const int units_per_tensor = hk * kPage * (kHeadDim * 2 / 16);   // 16 B units of one page, one tensor
-  const int units = 2 * units_per_tensor;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kUnits = kPage * kHeadDim * 2 / 16;            // 16-byte units of one (tensor, head) block
+  const int64_t block_units = kUnits;
+  const int64_t page_units = int64_t(hk) * kUnits;              // one page of one tensor, one layer
+  const int64_t layer_base = int64_t(p.layer) * p.num_pages;
   for (int i = blockIdx.x; i < n_cow; i += gridDim.x) {
     const int src = __ldcg(p.plan + p.lay.cow_src + i);
     const int dstp = __ldcg(p.plan + p.lay.cow_dst + i);
@@ -212,28 +218,23 @@ __global__ void __launch_bounds__(kRcCopyThreads) rc_copy_kernel(const RcCopyPar
       if (threadIdx.x == 0) atomicOr(p.plan + kRcHdrErr, kDevErrPage);
       continue;
     }
-    for (int u0 = threadIdx.x; u0 < units; u0 += kRcCopyThreads * kRcCopyUnroll) {
-      uint4 v[kRcCopyUnroll];
-      uint4* to[kRcCopyUnroll];
+    for (int blk = warp; blk < 2 * hk; blk += kRcCopyThreads / 32) {
+      const int tensor = blk / hk, h = blk % hk;
+      const uint4* from = reinterpret_cast<const uint4*>(tensor ? p.pool_v : p.pool_k) +
+                          (layer_base + src) * page_units + h * block_units;
+      uint4* to = reinterpret_cast<uint4*>(tensor ? p.pool_v : p.pool_k) + (layer_base + dstp) * page_units +
+                  h * block_units;
+      uint4 v[kUnits / 32];
 #pragma unroll
-      for (int j = 0; j < kRcCopyUnroll; ++j) {
-        const int u = u0 + j * kRcCopyThreads;
-        to[j] = nullptr;
-        if (u >= units) continue;
-        const int tensor = u / units_per_tensor;
-        const int rem = u % units_per_tensor;       // (head, slot, 16-byte column)
-        const int slot = (rem >> 4) & (kPage - 1);
-        if (mask & (1u << slot)) continue;
-        uint8_t* pool = tensor ? p.pool_v : p.pool_k;
-        const int64_t page_bytes = int64_t(hk) * kPage * kHeadDim * 2;
-        const int64_t layer_base = int64_t(p.layer) * p.num_pages;
-        const uint4* from = reinterpret_cast<const uint4*>(pool + (layer_base + src) * page_bytes) + rem;
-        to[j] = reinterpret_cast<uint4*>(pool + (layer_base + dstp) * page_bytes) + rem;
-        v[j] = __ldg(from);
+      for (int j = 0; j < kUnits / 32; ++j) {
+        const int u = lane + 32 * j;                            // slot u / 16
+        if (!(mask & (1u << (u >> 4)))) v[j] = __ldg(from + u);
       }
 #pragma unroll
-      for (int j = 0; j < kRcCopyUnroll; ++j)
-        if (to[j]) *to[j] = v[j];
+      for (int j = 0; j < kUnits / 32; ++j) {
+        const int u = lane + 32 * j;
+        if (!(mask & (1u << (u >> 4)))) to[u] = v[j];
+      }
     }
   }
 }
@@ -241,12 +242,13 @@ __global__ void __launch_bounds__(kRcCopyThreads) rc_copy_kernel(const RcCopyPar
 // ---------------------------------------------------------------- GEMM
 
 constexpr int kRcBM = 128;            // selected tokens per tile (MMA M, TMEM lanes)
-constexpr int kRcBN = 128;            // output columns per tile: one KV head of K or V
+constexpr int kRcHead = 128;          // output columns of one KV head
+constexpr int kRcBNMax = 2 * kRcHead; // output columns per tile: one or two heads of K or V
 constexpr int kRcBK = 64;             // hidden features per stage (128 B rows, 128B swizzle)
-constexpr int kRcStages = 6;
+constexpr int kRcStages = 4;
 constexpr int kRcABytes = kRcBM * kRcBK * 2;
-constexpr int kRcBBytes = kRcBN * kRcBK * 2;
-constexpr int kRcStageBytes = kRcABytes + kRcBBytes;
+constexpr int kRcBBytesMax = kRcBNMax * kRcBK * 2;
+constexpr int kRcStageBytes = kRcABytes + kRcBBytesMax;
 constexpr int kRcThreads = 192;       // producer, MMA, 4 epilogue warps
 
 struct RcCtrl {
@@ -282,7 +284,7 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, 256);
+    tmem_alloc(&ctl->tmem_base, 2 * kRcBNMax);   // two accumulators of up to 256 columns
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -295,7 +297,9 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
   int32_t* err = p.plan + kRcHdrErr;
   const int n_tok = __ldcg(p.plan + kRcHdrTok);
-  const int n_nt = 2 * p.num_kv_heads;
+  const int hpt = p.heads_per_tile;            // 1 or 2: an output tile is hpt heads of K or of V
+  const int bn = kRcHead * hpt;
+  const int n_nt = 2 * p.num_kv_heads / hpt;
   const int n_tiles = ((n_tok + kRcBM - 1) / kRcBM) * n_nt;
   const int nk = p.d_model / kRcBK;
   const uint32_t tmem = ctl->tmem_base;
@@ -321,8 +325,9 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int x = t < n_tok ? __ldcg(x_row + t) : -1;
         r[i] = (x < 0 || x >= p.x_rows) ? 0 : x;   // skipped rows read row 0; the epilogue stores nothing for them
       }
-      const CUtensorMap* tb = nt < p.num_kv_heads ? &tm_wk : &tm_wv;
-      const int brow = (nt % p.num_kv_heads) * kRcBN;
+      const int h0 = nt * hpt;                 // first output head, over K heads then V heads
+      const CUtensorMap* tb = h0 < p.num_kv_heads ? &tm_wk : &tm_wv;
+      const int brow = (h0 % p.num_kv_heads) * kRcHead;
       for (int ks = 0; ks < nk; ++ks, ++it) {
         const int s = it % kRcStages;
         if (it >= uint32_t(kRcStages) && !mbar_wait(&ctl->empty[s], ((it / kRcStages) - 1) & 1, abort_flag)) {
@@ -330,7 +335,7 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
           break;
         }
         uint8_t* sa = smem + s * kRcStageBytes;
-        if (lane == 0) mbar_arrive_expect_tx(&ctl->full[s], kRcStageBytes);
+        if (lane == 0) mbar_arrive_expect_tx(&ctl->full[s], kRcABytes + bn * kRcBK * 2);
         __syncwarp();
         if (tiled) {
           // rows past x_rows are filled with zeros; the epilogue stores nothing for them
@@ -353,14 +358,14 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kRcBM, kRcBN, 0);
+      const uint32_t idesc = idesc_bf16_f32(kRcBM, kRcHead * p.heads_per_tile, 0);
       uint32_t it = 0, tcount = 0;
       int bad = 0;
       for (int tile = blockIdx.x; tile < n_tiles && !bad; tile += gridDim.x, ++tcount) {
         const uint32_t buf = tcount & 1;
         if (tcount >= 2 && !mbar_wait(&ctl->acc_empty[buf], ((tcount - 2) >> 1) & 1, abort_flag)) { bad = 1; break; }
         tc_fence_after();
-        const uint32_t d = tmem + buf * kRcBN;
+        const uint32_t d = tmem + buf * kRcBNMax;
         for (int ks = 0; ks < nk; ++ks, ++it) {
           const int s = it % kRcStages;
           if (!mbar_wait(&ctl->full[s], (it / kRcStages) & 1, abort_flag)) { bad = 1; break; }
@@ -390,33 +395,36 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
       tc_fence_after();
       const int m0 = (tile / n_nt) * kRcBM;
       const int nt = tile % n_nt;
-      float acc[kRcBN];
-#pragma unroll
-      for (int c = 0; c < kRcBN / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_off + buf * kRcBN + 32 * c, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[32 * c + j] = __uint_as_float(u[j]);
-      }
-      tc_fence_before();
-      mbar_arrive(&ctl->acc_empty[buf]);
       const int t = m0 + row;
       const int xr = t < n_tok ? __ldcg(x_row + t) : -1;
-      if (xr >= 0) {
-        const int dv = __ldcg(dst + t);
-        const int page = dv / kPage, slot = dv % kPage;
-        if (xr >= p.x_rows) {
-          atomicOr(err, kDevErrGeometry);
-        } else if (page < 0 || page >= p.num_pages) {
-          atomicOr(err, kDevErrPage);
-        } else {
-          const int head = nt % p.num_kv_heads;
-          __nv_bfloat16* pool = nt < p.num_kv_heads ? p.pool_k : p.pool_v;
+      const int dv = xr >= 0 ? __ldcg(dst + t) : 0;
+      const int page = dv / kPage, slot = dv % kPage;
+      const bool store = xr >= 0 && xr < p.x_rows && page >= 0 && page < p.num_pages;
+      if (xr >= p.x_rows) atomicOr(err, kDevErrGeometry);
+      else if (xr >= 0 && (page < 0 || page >= p.num_pages)) atomicOr(err, kDevErrPage);
+      // one KV head (128 columns) at a time: read from TMEM, round, store
+      for (int hh = 0; hh < hpt; ++hh) {
+        float acc[kRcHead];
+#pragma unroll
+        for (int c = 0; c < kRcHead / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_off + buf * kRcBNMax + hh * kRcHead + 32 * c, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[32 * c + j] = __uint_as_float(u[j]);
+        }
+        if (hh == hpt - 1) {
+          tc_fence_before();
+          mbar_arrive(&ctl->acc_empty[buf]);   // the accumulator is read: the next tile may overwrite it
+        }
+        if (store) {
+          const int ho = nt * hpt + hh;       // output head over K heads then V heads
+          const int head = ho % p.num_kv_heads;
+          __nv_bfloat16* pool = ho < p.num_kv_heads ? p.pool_k : p.pool_v;
           const int64_t orow = ((int64_t(p.layer) * p.num_pages + page) * p.num_kv_heads + head) * kPage + slot;
           uint4* out = reinterpret_cast<uint4*>(pool + orow * kHeadDim);
 #pragma unroll
-          for (int c = 0; c < kRcBN / 8; ++c) {
+          for (int c = 0; c < kRcHead / 8; ++c) {
             uint4 v;
             v.x = pack_bf16x2(acc[8 * c + 0], acc[8 * c + 1]);
             v.y = pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]);
@@ -434,7 +442,7 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 2 * kRcBNMax);
   }
 }
 

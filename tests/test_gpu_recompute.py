@@ -38,6 +38,9 @@ def cases():
         # several 128-token tiles of selected tokens with a ragged tail, a long K loop
         "tiles": scaled(l3, num_layers=2, num_q_heads=16, num_kv_heads=4, chunk_lens=(700, 333, 901), q_len=20,
                         d_model=1024),
+        # an odd number of KV heads: output tiles of one head instead of two
+        "odd_heads": scaled(b16, num_q_heads=6, num_kv_heads=3, n_requests=3, n_pool_chunks=6,
+                            chunk_len_range=(20, 300), chunks_per_req=(1, 3), q_range=(1, 20), d_model=192),
     }
 
 
@@ -103,7 +106,7 @@ def assert_pool_matches(ref_plan, ref_bits, got_bits):
         assert (err <= bound).all(), f"recomputed rows: worst ratio {(err / bound).max():.3g}"
 
 
-@pytest.mark.parametrize("name", ["pooled", "tiles"])
+@pytest.mark.parametrize("name", ["pooled", "tiles", "odd_heads"])
 @pytest.mark.parametrize("by_selection", [False, True])
 def test_recompute_matches_oracle(name, by_selection):
     w = cases()[name]
