@@ -100,11 +100,19 @@ def _code_only(text: str) -> str:
     return "\n".join(lines)
 
 
-def kernel_sources_digest():
+# the source file of each timed kernel kind; its digest also covers the
+# device-side headers every kernel includes
+KERNEL_SOURCE = {"attn": "attn_fwd.cu", "combine": "attn_fwd.cu", "impact": "impact.cu", "topk": "topk.cu",
+                 "rc_gemm": "recompute.cu", "rc_copy": "recompute.cu", "rc_plan": "recompute.cu",
+                 "kv_decode": "kv_decode.cu", "simt_attn": "simt_f32.cu", "simt_impact": "simt_f32.cu"}
+
+
+def kernel_sources_digest(kernel, read=None):
+    """Digest of a kernel's source and the device headers, comments and blank lines removed."""
+    read = read or (lambda f: open(os.path.join(ROOT, "serving_prefill_b200", "csrc", f)).read())
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "serving_prefill_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        h.update(_code_only(open(os.path.join(csrc, f)).read()).encode())
+    for f in ("ptx.cuh", "common.cuh", KERNEL_SOURCE.get(kernel, "attn_fwd.cu")):
+        h.update(_code_only(read(f)).encode())
     return h.hexdigest()[:16]
 
 
@@ -115,7 +123,7 @@ def recorded_traffic(config, kernel):
         return None
     j = json.load(open(p))
     e = j.get(f"{config}/{kernel}")
-    if not e or e.get("src_digest") != kernel_sources_digest():
+    if not e or e.get("src_digest") != kernel_sources_digest(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -896,6 +904,8 @@ def main():
                     help="profiling mode: one input copy, eager launches, W + K steps, no JSON")
     ap.add_argument("--ncu-path", default="step", choices=["step", "recompute", "kv_decode"],
                     help="with --ncu: the fused step, the selective recompute or the KV decode")
+    ap.add_argument("--path", default="step", choices=["step", "recompute", "kv_decode"],
+                    help="time the selective recompute or the KV decode alone (one JSON line)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     w = get_workload(args.config)
@@ -927,6 +937,14 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     device = local
+    if args.path != "step" and not args.ncu:
+        # one of the further paths alone, timed like its per_config entry
+        run = run_recompute if args.path == "recompute" else run_kv_decode
+        wp = get_workload(RECOMPUTE_CONFIG if args.path == "recompute" else DECODE_CONFIG)
+        entry = run(args, wp, device, not args.no_cpu_baseline)
+        entry.update({"n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True})
+        print(json.dumps(entry))
+        return
     if args.ncu and args.ncu_path != "step":
         run = run_recompute if args.ncu_path == "recompute" else run_kv_decode
         st = run(args, w, device, False, ncu=True)
