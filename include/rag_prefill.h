@@ -73,9 +73,9 @@ typedef enum {
   RAG_ERR_TIMEOUT = 6,     /* device: a pipeline wait gave up                 */
   RAG_ERR_WORKSPACE = 7,   /* workspace missing or smaller than required      */
   RAG_ERR_GEOMETRY = 8,    /* device: chunk pages do not match its length     */
-  RAG_ERR_RANGE = 9,       /* device: a bf16 V value of magnitude >= 65536
-                              (or inf/nan) met the fp16 PV product and was
-                              saturated to +-65504; O is then inexact        */
+  RAG_ERR_RANGE = 9,       /* device: a V value of magnitude >= 65536 (or
+                              inf/nan) was stored or used as fp16 and was
+                              saturated to +-65504 (nan kept)                */
   RAG_ERR_NO_FREE_PAGES = 10 /* device: the copy-on-write recompute needs more
                               private pages than the free list holds          */
 } rag_status;
@@ -83,8 +83,15 @@ typedef enum {
 typedef enum { RAG_BF16 = 0, RAG_F32 = 1 } rag_dtype;
 
 /* The paged pool of precomputed chunk caches (caller-owned device memory).
- * k, v: [num_layers][num_pages][num_kv_heads][16][head_dim] of `dtype`.
+ * k, v: [num_layers][num_pages][num_kv_heads][16][head_dim].
  * Page p of layer l, kv head g holds 16 consecutive tokens of one chunk.
+ * Element types: RAG_F32 keeps K and V in fp32. RAG_BF16 (a bf16 cache)
+ * keeps K in bf16 and V in fp16, the type in which V enters the product
+ * with the attention weights. rag_kv_pool_write stores the fp16 value of each
+ * bf16 V value (exact for magnitudes in [2^-14, 65280], within 2^-25 below);
+ * rag_kv_decode and rag_recompute_kv round their fp32 V values once to fp16.
+ * All round to nearest even; magnitudes beyond the fp16 range, inf and nan
+ * saturate to +-65504 (nan kept) and the writing call reports RAG_ERR_RANGE.
  * Supported: RAG_BF16 with head_dim 128 (tensor-core path), RAG_F32 with
  * head_dim 64 or 128 (CUDA-core path). */
 typedef struct {
@@ -138,12 +145,13 @@ RAG_API int32_t rag_num_sms(void);
 
 /* Pool write (TurboRAG page, "Technical Details / KV cache precompute"; the
  * listing `precompute_kv_cache`): store one chunk's dense K, V
- * [n_tokens][num_kv_heads][head_dim] (pool dtype, device) into the pages
- * page_ids[0 .. n_pages-1] (device int32) of `layer`. Token t goes to page
- * page_ids[t / 16], slot t % 16; the slots of the last page beyond n_tokens
- * are zeroed. n_pages must equal ceil(n_tokens / 16). A page id outside the
- * pool is skipped and sets RAG_ERR_PAGE_OOB's bit in *device_err (optional
- * device int32, may be NULL). */
+ * [n_tokens][num_kv_heads][head_dim] (pool dtype: bf16 or fp32, device) into
+ * the pages page_ids[0 .. n_pages-1] (device int32) of `layer`. Token t goes
+ * to page page_ids[t / 16], slot t % 16; the slots of the last page beyond
+ * n_tokens are zeroed. n_pages must equal ceil(n_tokens / 16). In a bf16 pool
+ * V is stored as fp16 (see rag_kv_pool). *device_err (optional device int32,
+ * may be NULL) collects bits: 1 a page id outside the pool (skipped), 8 a V
+ * value saturated. */
 RAG_API rag_status rag_kv_pool_write(const rag_kv_pool* pool, int32_t layer, const int32_t* page_ids, int32_t n_pages,
                              int32_t n_tokens, const void* k, const void* v, int32_t* device_err, void* stream);
 
@@ -176,10 +184,11 @@ RAG_API rag_status rag_workspace_init(void* workspace, size_t workspace_bytes, v
  *   Pass it on the layer whose attention selects tokens (the last layer).
  * workspace: device, >= rag_workspace_size() bytes, 256-byte aligned.
  * Precision (bf16 pool): scores and the softmax run in fp32; the PV product
- * takes P and V in fp16, which holds every bf16 V value of magnitude up to
- * 65280 (below 2^-14 with an absolute error under 2^-24). A V value of
- * magnitude 65536 or more (or inf/nan) is saturated to +-65504 and the call
- * reports RAG_ERR_RANGE through rag_last_device_error. */
+ * takes the weights P and V in fp16 (P keeps 3 more mantissa bits than bf16)
+ * with an fp32 accumulator. The pool holds V as fp16 already; the query
+ * block's vq (bf16) is rounded to fp16 the same way, and a vq value of
+ * magnitude 65536 or more (or inf/nan) is saturated and the call reports
+ * RAG_ERR_RANGE through rag_last_device_error. */
 RAG_API rag_status rag_fused_prefill_attn(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch, const void* q,
                                   int32_t num_q_heads, const void* kq, const void* vq, float sm_scale, void* o,
                                   float* row_lse, float* impact, void* workspace, size_t workspace_bytes,
@@ -263,7 +272,8 @@ RAG_API rag_status rag_impact_topk(const float* impact, const rag_batch* batch, 
  * give no stream format; this entry point decodes the plainest one they
  * support: per chunk, layer, KV head and channel, b-bit codes (b = 8 or 4,
  * chosen per call, i.e. per layer) of a uniform quantization with an fp32
- * scale and offset. value = fp32 fma(code, scale, offset), stored as bf16.
+ * scale and offset. value = fp32 fma(code, scale, offset), rounded once to
+ * the type the pool stores it in (bf16 for K, fp16 for V, see rag_kv_pool).
  *
  * One call decodes n_chunks chunks of one layer (bf16 pool, head_dim 128):
  *   chunk_tok_off  [n_chunks+1] device int32: token prefix over the chunks
@@ -277,7 +287,8 @@ RAG_API rag_status rag_impact_topk(const float* impact, const rag_batch* batch, 
  * Token t of chunk c lands in slot t % 16 of page page_ids[chunk_page_off[c] +
  * t / 16]; the last page's slots past the chunk are zeroed. A page id outside
  * the pool or a chunk whose page count is not ceil(n_c / 16) is skipped and
- * recorded in *device_err (optional device int32: 1 page, 2 geometry). */
+ * recorded in *device_err (optional device int32: 1 page, 2 geometry, 8 a V
+ * value saturated). */
 RAG_API rag_status rag_kv_decode(const rag_kv_pool* pool, int32_t layer, int32_t n_chunks,
                                  const int32_t* chunk_tok_off, const int32_t* chunk_page_off,
                                  const int32_t* page_ids, int32_t total_pages, int32_t bits, const void* codes_k,
@@ -329,14 +340,16 @@ RAG_API rag_status rag_recompute_plan(const rag_batch* batch, const int32_t* top
  *   every private page first receives, for this layer, the K and V of every
  *   slot that is not selected from the page it replaces (all KV heads);
  *   every selected token's rows are recomputed from its hidden state:
- *   K = x W_K^T, V = x W_V^T (fp32 accumulation, one rounding to bf16), split
- *   into num_kv_heads heads of 128, and stored into its slot of its private
- *   page. The copy and the recompute never write the same bytes.
+ *   K = x W_K^T, V = x W_V^T (fp32 accumulation, one rounding to the stored
+ *   type: bf16 for K, fp16 for V, see rag_kv_pool), split into num_kv_heads
+ *   heads of 128, and stored into its slot of its private page. The copy
+ *   and the recompute never write the same bytes.
  * x   [x_rows][d_model] bf16 device, rows as x_by_selection of the plan says;
  * w_k, w_v [num_kv_heads * 128][d_model] bf16 device (a linear layer's weight);
  * d_model a multiple of 64. batch and k_cap as given to rag_recompute_plan.
  * Device problems (a free page id outside the pool, a row past x_rows, a wait
- * that gave up) are recorded in the plan and reported by rag_recompute_status. */
+ * that gave up, a V value saturated) are recorded in the plan and reported by
+ * rag_recompute_status. */
 RAG_API rag_status rag_recompute_kv(const rag_kv_pool* pool, int32_t layer, const rag_batch* batch, int32_t k_cap,
                                     const void* plan, size_t plan_bytes, const void* x, int64_t x_rows,
                                     int32_t d_model, const void* w_k, const void* w_v, void* stream);

@@ -21,9 +21,11 @@ give no stream format. This restatement takes the plainest reading of that:
   stored channel by channel; with 4 bits two channels share a byte, the even
   channel in the low nibble.
 * Decoding: v = fp32(code * scale + offset) (one fused multiply-add, one
-  rounding to fp32), stored in the pool dtype (bf16, round to nearest even),
-  token t of the chunk in page page_ids[t // 16], slot t % 16; the slots of
-  the last page past the chunk's end are zeroed (as the pool write does).
+  rounding to fp32), rounded once more to the type the pool stores it in (a
+  bf16 cache keeps K in bf16 and V in fp16; round to nearest even, V
+  saturated beyond 65504), token t of the chunk in page page_ids[t // 16],
+  slot t % 16; the slots of the last page past the chunk's end are zeroed (as
+  the pool write does).
 
 The entropy coding of the real system is not described by the pages and is
 not part of this restatement.
@@ -35,6 +37,8 @@ from dataclasses import dataclass
 
 import numpy as np
 import torch
+
+from .prefill import f16_bits_sat
 
 PAGE_SIZE = 16
 
@@ -110,11 +114,12 @@ def to_bf16_bits(x32: np.ndarray) -> np.ndarray:
 
 def decode_into_pool(pool_k: np.ndarray, pool_v: np.ndarray, layer: int, page_ids, enc: EncodedChunk,
                      n_tokens: int) -> None:
-    """Decode one chunk of one layer into its pages (bf16 bits pools [L][pages][H_kv][16][d])."""
+    """Decode one chunk of one layer into its pages (pools [L][pages][H_kv][16][d]
+    of a bf16 cache: K bf16 bits, V fp16 bits)."""
     ck = unpack(enc.codes_k, enc.bits)
     cv = unpack(enc.codes_v, enc.bits)
     kb = to_bf16_bits(dequantize_f32(ck, enc.scale_k[None], enc.offset_k[None]))
-    vb = to_bf16_bits(dequantize_f32(cv, enc.scale_v[None], enc.offset_v[None]))
+    vb = f16_bits_sat(dequantize_f32(cv, enc.scale_v[None], enc.offset_v[None]).astype(np.float64))
     page_ids = np.asarray(page_ids, dtype=np.int64)
     assert len(page_ids) == -(-n_tokens // PAGE_SIZE)
     for t in range(n_tokens):

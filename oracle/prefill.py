@@ -12,7 +12,13 @@ What it computes, step by step, in the pages' order:
    pool [layers][pages][H_kv][16][d]. The page layout is this library's choice
    (the TurboRAG page's related-work section points at PagedAttention); each
    chunk starts on a fresh page and the unused tail slots of its last page are
-   zero.
+   zero. The storage format is this library's choice too (the pages fix no
+   precision): in a bf16 cache, K is stored as bf16 and V as the fp16 value of
+   its bf16 value (round to nearest even; magnitudes beyond 65504 saturate),
+   the operand type in which V enters the product with the normalised
+   weights. Every bf16 value of magnitude in [2^-14, 65280] is exact in fp16;
+   smaller ones move by less than 2^-25. The query block's own V_q enters the
+   product in the same form.
 2. Concat (TurboRAG page, "Technical Details", K_combined = Concat(K^(1), ...,
    K^(m), K^(Q)); CacheBlend page, "Mathematical formulation",
    K_concat = [K_1; ...; K_m; K_q]): the request's chunks in retrieval order
@@ -72,6 +78,28 @@ def bits_to_f64(b: np.ndarray) -> np.ndarray:
 
 def to_f64(t: torch.Tensor) -> np.ndarray:
     return t.to(torch.float64).numpy()
+
+
+F16_MAX = 65504.0
+
+
+def f16_bits_sat(x: np.ndarray) -> np.ndarray:
+    """fp64 values -> fp16 bits, rounded once to nearest (ties to even),
+    magnitudes beyond 65504 (inf included) saturated to +-65504, nan kept."""
+    x = np.asarray(x, dtype=np.float64)
+    x = np.where(np.isnan(x), x, np.clip(x, -F16_MAX, F16_MAX))
+    return x.astype(np.float16).view(np.uint16)
+
+
+def v_operand_bits(b: np.ndarray) -> np.ndarray:
+    """Stored V of a bf16 cache: bf16 bits -> fp16 bits of the same value
+    (f16_bits_sat of the exact bf16 value)."""
+    return f16_bits_sat(bits_to_f64(b))
+
+
+def f16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    """Exact fp64 value of fp16 bits."""
+    return np.asarray(b, dtype=np.uint16).view(np.float16).astype(np.float64)
 
 
 # --------------------------------------------------------------------------
@@ -253,7 +281,7 @@ class OracleResult:
     k: list = field(default_factory=list)
     topk: list = field(default_factory=list)   # per request: int64 positions
     pool_k: np.ndarray = None          # raw bits [1, pages, H_kv, 16, d] of this layer
-    pool_v: np.ndarray = None
+    pool_v: np.ndarray = None          # (V of a bf16 cache: fp16 bits)
 
 
 def build_layer_pool(lay, inputs, bits_dtype):
@@ -261,9 +289,15 @@ def build_layer_pool(lay, inputs, bits_dtype):
     pk = new_pool(1, lay.num_pages, w.num_kv_heads, w.head_dim, bits_dtype)
     pv = new_pool(1, lay.num_pages, w.num_kv_heads, w.head_dim, bits_dtype)
     for c, pages in enumerate(lay.chunk_pages):
+        vb = to_bits(inputs.chunk_v[c])
         pool_write(pk, 0, pages.numpy(), to_bits(inputs.chunk_k[c]))
-        pool_write(pv, 0, pages.numpy(), to_bits(inputs.chunk_v[c]))
+        pool_write(pv, 0, pages.numpy(), v_operand_bits(vb) if bits_dtype == np.uint16 else vb)
     return pk, pv
+
+
+def v_values(bits: np.ndarray) -> np.ndarray:
+    """Exact values of stored V bits: fp16 in a bf16 cache, fp32 in an fp32 one."""
+    return f16_bits_to_f64(bits) if bits.dtype == np.uint16 else bits_to_f64(bits)
 
 
 def run_workload_layer(lay, inputs, want_impact: bool, scale: float = None,
@@ -277,7 +311,8 @@ def run_workload_layer(lay, inputs, want_impact: bool, scale: float = None,
     pk, pv = build_layer_pool(lay, inputs, bits_dtype)
     q_all = to_f64(inputs.q)
     kq_all = to_f64(inputs.kq)
-    vq_all = to_f64(inputs.vq)
+    vq_bits = to_bits(inputs.vq)
+    vq_all = v_values(v_operand_bits(vq_bits) if bits_dtype == np.uint16 else vq_bits)
     tq = lay.total_q
     o = np.zeros((tq, w.num_q_heads, d))
     m = np.zeros((tq, w.num_q_heads))
@@ -293,7 +328,7 @@ def run_workload_layer(lay, inputs, want_impact: bool, scale: float = None,
             if bits_dtype != np.uint16:
                 raise TypeError("re-basing is defined for bf16 caches")
             kd = bits_to_f64(gather_rebased(pk, 0, chunks, rope_base))
-        vd = bits_to_f64(gather(pv, 0, chunks))
+        vd = v_values(gather(pv, 0, chunks))
         n_doc = kd.shape[0]
         kcat = np.concatenate([kd, kq_all[q0:q0 + ql]], axis=0)
         vcat = np.concatenate([vd, vq_all[q0:q0 + ql]], axis=0)

@@ -25,8 +25,9 @@ values -> generate from the fused cache):
    token's K and V rows are recomputed from its hidden state x (the layer's
    input for that token): K = x W_K^T, V = x W_V^T, with W_K, W_V of shape
    [H_kv * d, d_model] (a linear layer's weight), split into H_kv heads of d,
-   rounded once to the pool dtype (bf16, round to nearest even), and stored
-   in the token's slot of its private page.
+   rounded once to the type the pool stores it in (a bf16 cache keeps K in
+   bf16 and V in fp16; round to nearest even, V saturated beyond 65504), and
+   stored in the token's slot of its private page.
 
 The hidden states are gathered per selected token either by its doc position
 (row doc_start_b + i of a [total_doc, d_model] array) or by its rank in the
@@ -41,6 +42,8 @@ from dataclasses import dataclass
 
 import numpy as np
 import torch
+
+from .prefill import f16_bits_sat
 
 PAGE_SIZE = 16
 
@@ -120,7 +123,8 @@ def bits_to_f64(b: np.ndarray) -> np.ndarray:
 
 def apply(pool_k: np.ndarray, pool_v: np.ndarray, layer: int, p: RecomputePlan, x: np.ndarray,
           w_k: np.ndarray, w_v: np.ndarray) -> None:
-    """One layer of the recompute, in place on bf16-bit pools [L][pages][H_kv][16][d].
+    """One layer of the recompute, in place on the pools [L][pages][H_kv][16][d]
+    of a bf16 cache (K: bf16 bits, V: fp16 bits).
 
     x: hidden states (exact fp64 values of the bf16 inputs), rows as p.x_row
     names them; w_k, w_v: [H_kv * d, d_model] (fp64 values).
@@ -133,7 +137,7 @@ def apply(pool_k: np.ndarray, pool_v: np.ndarray, layer: int, p: RecomputePlan, 
         return
     xs = x[p.x_row]                                   # gather: one hidden state per selected token
     k_new = round_bf16_bits(xs @ w_k.T).reshape(len(p.x_row), hk, d)
-    v_new = round_bf16_bits(xs @ w_v.T).reshape(len(p.x_row), hk, d)
+    v_new = f16_bits_sat(xs @ w_v.T).reshape(len(p.x_row), hk, d)
     for t in range(len(p.x_row)):
         pool_k[layer, p.dst_page[t], :, p.dst_slot[t], :] = k_new[t]
         pool_v[layer, p.dst_page[t], :, p.dst_slot[t], :] = v_new[t]

@@ -11,7 +11,9 @@
 //   K producer warp : Q tiles, then page table -> 8 TMA page boxes per K tile
 //                     (or one box of K_q), and the tile's mask descriptor
 //   V producer warp : the same for V
-//   V converter warp: V tile bf16 -> fp16 in place (PV runs in fp16)
+//   convert warp    : the tile of the query block's own V_q (a bf16 input)
+//                     rounded to fp16 in place; with position re-basing, each
+//                     K tile rotated in place to its concatenated positions
 //   MMA warp        : S_i = Q_i K^T (tcgen05 smem x smem -> TMEM) for both Q
 //                     tiles, then O_i += P_i V (P_i from TMEM, V from smem)
 //   2 x 4 softmax warps: warpgroup i owns Q tile i; thread = row = TMEM lane;
@@ -19,6 +21,9 @@
 //                     written over the columns of S_i, lazy O_i rescale
 // The two softmax warpgroups alternate with the tensor core: while one
 // computes exponentials the MMA warp runs the other Q tile's products.
+// PV runs in fp16 (P and V): P keeps 3 more mantissa bits than bf16, and the
+// pool of a bf16 cache stores V as fp16 already, so doc V tiles go from TMA
+// to the tensor core untouched.
 // kPolyPairsOf8 can move a share of the exponentials onto the FMA pipe
 // (exp2_poly2); measured on B200 this pass runs fastest with all of them on
 // MUFU. Every wait is bounded; a timeout raises a device error instead of
@@ -595,23 +600,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     __syncwarp();
   } else if (warp == 11) {
-    // ------------------------------------------------------------ V converter
-    // The PV product runs in fp16 (P and V): P keeps 3 more mantissa bits than
-    // bf16, and every bf16 V value of magnitude in [2^-14, 65280] is exact in
-    // fp16 (smaller ones keep an absolute error below 2^-24). Magnitudes from
-    // 65536 up (and inf, nan) do not fit: they saturate, and the tile raises
-    // kDevErrRange. The tile is rewritten in place; the 128B swizzle is
-    // unchanged.
+    // ------------------------------------------------------------ convert warp
+    // Per tile, in order: with position re-basing, the K tile is rotated in
+    // place to the concatenated positions of its keys; then the V stage is
+    // released to the MMA warp (vconv), after rounding it from bf16 to fp16 in
+    // place when it holds the query block's own V_q (doc V tiles are fp16 in
+    // the pool already). Every bf16 V_q value of magnitude in [2^-14, 65280]
+    // is exact in fp16; magnitudes from 65536 up, inf and nan saturate and
+    // raise kDevErrRange. Rows past the request's query block are zeroed (a
+    // masked key must still hold a finite value). The 128B swizzle is
+    // unchanged by an elementwise rewrite.
     uint32_t t_glob = 0;
     int bad = 0;
-    uint32_t range = 0;   // bit 15 of a halfword: some |v| >= 65536 (bf16 0x4780)
+    uint32_t range = 0;
     for (int w = blockIdx.x; w < total_items && !bad; w += gridDim.x) {
       const FwdItem it = decode_fwd_item(p, prefix, w);
       const int n = it.t_end - it.t_begin;
       for (int i = 0; i < n; ++i) {
         const uint32_t t = t_glob + i;
+        const int tile = it.t_begin + i;
         if (p.rope) {
-          // re-base the cached keys of this K tile to their concatenated positions
           const int sk = t % kKStages;
           if (!mbar_wait(&ctl->kfull[sk], (t / kKStages) & 1, abort_flag)) { bad = 1; break; }
           rope_rotate_tile(sK + sk * kTileBytes, ctl->kchunk[sk], p.rope, lane);
@@ -621,28 +629,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         const int s = t % kVStages;
         if (!mbar_wait(&ctl->vfull[s], (t / kVStages) & 1, abort_flag)) { bad = 1; break; }
-        uint4* tile = reinterpret_cast<uint4*>(sV + s * kTileBytes);
+        if (tile >= it.n_doc_tiles) {
+          const int rows = min(kBN, it.req.n_q - (tile - it.n_doc_tiles) * kBN);
+          uint8_t* base = sV + s * kTileBytes;
 #pragma unroll 4
-        for (int v = lane; v < kTileBytes / 16; v += 32) {
-          uint4 x = tile[v];
-          // |h| + 0x3880 reaches 0x8000 exactly when |h| >= 0x4780; no carry
-          // crosses into the other halfword
-          range |= ((x.x & 0x7fff7fffu) + 0x38803880u) | ((x.y & 0x7fff7fffu) + 0x38803880u) |
-                   ((x.z & 0x7fff7fffu) + 0x38803880u) | ((x.w & 0x7fff7fffu) + 0x38803880u);
-          x.x = bf16x2_to_f16x2(x.x);
-          x.y = bf16x2_to_f16x2(x.y);
-          x.z = bf16x2_to_f16x2(x.z);
-          x.w = bf16x2_to_f16x2(x.w);
-          tile[v] = x;
+          for (int u = lane; u < kBN * (kHeadDim / 8); u += 32) {
+            const int r = u >> 4, c = u & 15;   // row, 16-byte chunk of the row
+            uint4* at = reinterpret_cast<uint4*>(base + (c >> 3) * kHalfBytes + r * 128 + ((c & 7) << 4));
+            *at = r < rows ? bf16x8_to_f16x8(*at, range) : make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->vconv[s]);
       }
       t_glob += n;
     }
     if (bad) raise_abort(ctl, p.err);
-    if (__any_sync(0xffffffffu, (range & 0x80008000u) != 0) && lane == 0) atomicOr(p.err, kDevErrRange);
+    if (range_exceeded(range)) atomicOr(p.err, kDevErrRange);
     __syncwarp();
   } else {
     // ------------------------------------------------------------ MMA issuer (warp 10)
@@ -684,7 +688,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t t = t_glob + i;
             const int sv = t % kVStages;
             const int b = i & 1;
-            if (!mbar_wait(&ctl->vconv[sv], (t / kVStages) & 1, abort_flag)) { bad = 1; break; }
+            // doc V tiles straight from TMA; the V_q tile once it is fp16
+            const bool v_doc = it.t_begin + i < it.n_doc_tiles;
+            if (!mbar_wait(v_doc ? &ctl->vfull[sv] : &ctl->vconv[sv], (t / kVStages) & 1, abort_flag)) {
+              bad = 1;
+              break;
+            }
             if (i == 0) {
               if (n_item[0] > 0 && !mbar_wait(&ctl->o_free[0], (n_item[0] - 1) & 1, abort_flag)) { bad = 1; break; }
               ++n_item[0];
@@ -718,17 +727,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const uint32_t tp = t - 1;              // tile of the PV products of this step
           const int s = t % kKStages;
           const int sv = tp % kVStages;
-          uint32_t v_base = 0, k_base = 0;
+          uint32_t v_base = 0;
+          const uint32_t k_base = smem_u32(sK + s * kTileBytes);
           if (i >= 1) {
-            if (!mbar_wait(&ctl->vconv[sv], (tp / kVStages) & 1, abort_flag)) { bad = 1; break; }
-            v_base = smem_u32(sV + sv * kTileBytes);
-          }
-          if (i < n) {
-            if (!mbar_wait(p.rope ? &ctl->kconv[s] : &ctl->kfull[s], (t / kKStages) & 1, abort_flag)) {
+            const bool v_doc = it.t_begin + i - 1 < it.n_doc_tiles;
+            if (!mbar_wait(v_doc ? &ctl->vfull[sv] : &ctl->vconv[sv], (tp / kVStages) & 1, abort_flag)) {
               bad = 1;
               break;
             }
-            k_base = smem_u32(sK + s * kTileBytes);
+            v_base = smem_u32(sV + sv * kTileBytes);
           }
           for (int q = 0; q < it.n_qt && !bad; ++q) {
             if (i >= 1) {
@@ -754,8 +761,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               ++npf;
               tc_commit(&ctl->pv_done[q]);
               if (i == n) tc_commit(&ctl->o_full[q]);   // O_q of this item is complete
+              if (q == it.n_qt - 1) tc_commit(&ctl->vempty[sv]);   // the last read of this V stage
             }
             if (i < n) {
+              // K of this tile is waited for only here, so that PV_0 of the
+              // previous tile never waits on the next tile's load
+              if (q == 0 &&
+                  !mbar_wait(p.rope ? &ctl->kconv[s] : &ctl->kfull[s], (t / kKStages) & 1, abort_flag)) {
+                bad = 1;
+                break;
+              }
               // S_q = Q_q K^T for this tile. It overwrites P_q (aliased over S_q),
               // which PV_q of the previous tile reads: tcgen05.mma operations of
               // one CTA execute in issue order, so no completion wait is needed.
@@ -768,7 +783,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
           }
           if (bad) break;
-          if (i >= 1) tc_commit(&ctl->vempty[sv]);
           if (i < n) tc_commit(&ctl->kempty[s]);
           // the drain step reads no Q: the next item's Q may load now
           if (i == n - 1) tc_commit(&ctl->q_empty);

@@ -25,7 +25,7 @@ enum : int32_t {
   kDevErrPage = 1,       // a page id outside [0, num_pages)
   kDevErrGeometry = 2,   // a chunk whose page count is not ceil(len / 16)
   kDevErrTimeout = 4,    // a pipeline wait gave up
-  kDevErrRange = 8,      // a V value beyond the fp16 range was saturated in the PV product
+  kDevErrRange = 8,      // a V value beyond the fp16 range was saturated when stored as fp16
 };
 
 struct BatchDev {

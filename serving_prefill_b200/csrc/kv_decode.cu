@@ -7,8 +7,10 @@
 // Stream of one chunk, one layer: per token and KV head, head_dim codes of b
 // bits (b = 8: one byte per channel; b = 4: two channels per byte, the even
 // channel in the low nibble), with one fp32 (scale, offset) per KV head and
-// channel. Value = fp32 fma(code, scale, offset), stored as bf16 in slot
-// t % 16 of page page_ids[t / 16]; slots past the chunk's end are zeroed.
+// channel. Value = fp32 fma(code, scale, offset), rounded once to the type the
+// pool stores it in (K bf16, V fp16: nearest even, V saturated beyond 65504
+// with kDevErrRange raised) and stored in slot t % 16 of page page_ids[t / 16];
+// slots past the chunk's end are zeroed.
 //
 // One CTA per page of the batch: 16 slots x H_kv heads x 128 channels for K
 // and for V; a thread makes 8 channels of one head (16-byte stores) for all 16
@@ -22,7 +24,7 @@ namespace rag {
 
 constexpr int kDecThreads = 256;
 
-__global__ void __launch_bounds__(kDecThreads) kv_decode_kernel(const KvDecodeParams p) {
+__global__ void __launch_bounds__(kDecThreads, 4) kv_decode_kernel(const KvDecodeParams p) {
   // no early release: the attention kernel reads pool pages before its own
   // wait, so it must start only once every page written here is complete
   const int gp = blockIdx.x;   // page of the batch
@@ -54,6 +56,7 @@ __global__ void __launch_bounds__(kDecThreads) kv_decode_kernel(const KvDecodePa
   // A thread owns one (tensor, KV head, 8-channel group): its scale and offset
   // are loaded once, then the codes of all 16 slots are loaded before the
   // first value is computed (16 loads in flight), and 16 stores follow.
+  bool over = false;   // a V value saturated
   for (int u = threadIdx.x; u < 2 * hk * (kHeadDim / 8); u += kDecThreads) {
     const int tensor = u / (hk * (kHeadDim / 8));
     const int h = (u / (kHeadDim / 8)) % hk;
@@ -62,6 +65,18 @@ __global__ void __launch_bounds__(kDecThreads) kv_decode_kernel(const KvDecodePa
     const float4* scale = reinterpret_cast<const float4*>((tensor ? p.scale_v : p.scale_k) + so);
     const float4* offset = reinterpret_cast<const float4*>((tensor ? p.offset_v : p.offset_k) + so);
     const float4 s0 = __ldg(scale), s1 = __ldg(scale + 1), o0 = __ldg(offset), o1 = __ldg(offset + 1);
+    // A decoded value is linear in its code, and rounding is monotonic, so
+    // its magnitude is at most that of the ends, code 0 and code 2^b - 1: when
+    // both are within the fp16 range, no V value of the group is checked one
+    // by one (a nan scale or offset fails the test).
+    bool v_checked = false;
+    if (tensor) {
+      const float top = float((1 << p.bits) - 1);
+      const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      const float of[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v_checked = v_checked || beyond_f16(of[i]) || beyond_f16(__fmaf_rn(top, sc[i], of[i]));
+    }
     const uint8_t* codes = (tensor ? p.codes_v : p.codes_k) + (int64_t(t_first) * hk + h) * code_row;
     const int64_t token_stride = int64_t(hk) * code_row;
     uint2 cw[kPage];
@@ -89,14 +104,35 @@ __global__ void __launch_bounds__(kDecThreads) kv_decode_kernel(const KvDecodePa
 #pragma unroll
           for (int i = 0; i < 8; ++i) q[i] = float((cw[slot].x >> (4 * i)) & 0xfu);
         }
-        v.x = pack_bf16x2(__fmaf_rn(q[0], s0.x, o0.x), __fmaf_rn(q[1], s0.y, o0.y));
-        v.y = pack_bf16x2(__fmaf_rn(q[2], s0.z, o0.z), __fmaf_rn(q[3], s0.w, o0.w));
-        v.z = pack_bf16x2(__fmaf_rn(q[4], s1.x, o1.x), __fmaf_rn(q[5], s1.y, o1.y));
-        v.w = pack_bf16x2(__fmaf_rn(q[6], s1.z, o1.z), __fmaf_rn(q[7], s1.w, o1.w));
+        float y[8];
+        y[0] = __fmaf_rn(q[0], s0.x, o0.x);
+        y[1] = __fmaf_rn(q[1], s0.y, o0.y);
+        y[2] = __fmaf_rn(q[2], s0.z, o0.z);
+        y[3] = __fmaf_rn(q[3], s0.w, o0.w);
+        y[4] = __fmaf_rn(q[4], s1.x, o1.x);
+        y[5] = __fmaf_rn(q[5], s1.y, o1.y);
+        y[6] = __fmaf_rn(q[6], s1.z, o1.z);
+        y[7] = __fmaf_rn(q[7], s1.w, o1.w);
+        if (tensor) {
+          if (v_checked) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) over |= beyond_f16(y[i]);
+          }
+          v.x = pack_f16x2_sat(y[0], y[1]);
+          v.y = pack_f16x2_sat(y[2], y[3]);
+          v.z = pack_f16x2_sat(y[4], y[5]);
+          v.w = pack_f16x2_sat(y[6], y[7]);
+        } else {
+          v.x = pack_bf16x2(y[0], y[1]);
+          v.y = pack_bf16x2(y[2], y[3]);
+          v.z = pack_bf16x2(y[4], y[5]);
+          v.w = pack_bf16x2(y[6], y[7]);
+        }
       }
       out[slot * (kHeadDim / 8)] = v;
     }
   }
+  if (over && p.err) atomicOr(p.err, kDevErrRange);
 }
 
 cudaError_t launch_kv_decode(const KvDecodeParams& p, int total_pages, cudaStream_t stream) {

@@ -156,6 +156,7 @@ struct PoolWriteParams {
   int32_t* err;
   int32_t layer, num_pages, num_kv_heads, n_tokens;
   int32_t row_bytes;
+  int32_t v_to_f16;   // bf16 pool: V is stored as fp16 (its bf16 value, saturated beyond 65504)
 };
 
 // Selective recompute. The plan buffer (int32 words, each region 64-word

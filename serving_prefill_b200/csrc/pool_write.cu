@@ -6,6 +6,11 @@
 // page_ids[t / 16], slot t % 16. The slots of the last page past the chunk's
 // end are zeroed, so that a gathered tile holds only finite values.
 //
+// In a bf16 pool V is stored as fp16, the type in which it enters the product
+// with the normalised weights: each bf16 value is rounded to the nearest fp16
+// value (exact for magnitudes in [2^-14, 65280]); magnitudes from 65536 up,
+// inf and nan saturate (nan stays nan) and raise kDevErrRange.
+//
 // One CTA per (page, kv head); each thread moves one 16-byte vector, so a
 // 4 KB bf16 page row block is one fully coalesced read and write.
 #include <cuda_runtime.h>
@@ -27,6 +32,7 @@ __global__ void __launch_bounds__(256) pool_write_kernel(const PoolWriteParams p
   const int nvec = kPage * vec_per_row;
   const size_t dst_base =
       ((size_t(p.layer) * p.num_pages + page) * p.num_kv_heads + g) * kPage * size_t(p.row_bytes);
+  uint32_t range = 0;
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
     const int slot = v / vec_per_row;
     const int off = (v % vec_per_row) * 16;
@@ -37,10 +43,12 @@ __global__ void __launch_bounds__(256) pool_write_kernel(const PoolWriteParams p
       a = *reinterpret_cast<const uint4*>(p.k + src);
       c = *reinterpret_cast<const uint4*>(p.v + src);
     }
+    if (p.v_to_f16) c = bf16x8_to_f16x8(c, range);
     const size_t dst = dst_base + size_t(slot) * p.row_bytes + off;
     *reinterpret_cast<uint4*>(p.pool_k + dst) = a;
     *reinterpret_cast<uint4*>(p.pool_v + dst) = c;
   }
+  if (range_exceeded(range) && p.err) atomicOr(p.err, kDevErrRange);
 }
 
 cudaError_t launch_pool_write(const PoolWriteParams& p, int n_pages, cudaStream_t stream) {

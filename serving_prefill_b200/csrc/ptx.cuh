@@ -86,6 +86,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
+// Non-blocking test of a phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait for a single issuing thread on the critical path: polls without
+// suspending, so it reacts to the phase completing within a few cycles (a
+// suspended try_wait resumes later). Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t k = 1;; ++k) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((k & 255u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
@@ -268,9 +296,18 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
+// As pack_f16x2, with magnitudes beyond the fp16 range saturated to +-65504
+// (inf too; nan stays nan).
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Two bf16 values (one 32-bit word) to two fp16 values, same positions. Exact
-// for magnitudes in [2^-14, 65504]; smaller ones round to fp16 subnormals and
-// larger ones saturate to +-65504.
+// for magnitudes in [2^-14, 65280] (every such bf16 value is an fp16 value);
+// smaller ones round to fp16 subnormals (nearest, ties to even) and larger
+// ones saturate to +-65504.
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   const float lo = __uint_as_float(w << 16);
   const float hi = __uint_as_float(w & 0xffff0000u);
@@ -278,6 +315,26 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+
+// Eight bf16 values to eight fp16 values; `range` collects bit 15 of each
+// halfword of |h| + 0x3880, which is set exactly when |h| >= 0x4780 (a
+// magnitude of 65536 or more, inf or nan: the values that saturate). No carry
+// crosses into the other halfword.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 x, uint32_t& range) {
+  range |= ((x.x & 0x7fff7fffu) + 0x38803880u) | ((x.y & 0x7fff7fffu) + 0x38803880u) |
+           ((x.z & 0x7fff7fffu) + 0x38803880u) | ((x.w & 0x7fff7fffu) + 0x38803880u);
+  uint4 y;
+  y.x = bf16x2_to_f16x2(x.x);
+  y.y = bf16x2_to_f16x2(x.y);
+  y.z = bf16x2_to_f16x2(x.z);
+  y.w = bf16x2_to_f16x2(x.w);
+  return y;
+}
+
+__device__ __forceinline__ bool range_exceeded(uint32_t range) { return (range & 0x80008000u) != 0; }
+
+// True when an fp32 value rounds beyond the fp16 range (|x| >= 65520) or is nan.
+__device__ __forceinline__ bool beyond_f16(float x) { return !(fabsf(x) < 65520.f); }
 
 // Packed fp32 pair arithmetic (one instruction for two lanes of work).
 __device__ __forceinline__ uint64_t f2_bits(float2 v) {

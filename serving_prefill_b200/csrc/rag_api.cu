@@ -284,6 +284,7 @@ rag_status rag_kv_pool_write(const rag_kv_pool* pool, int32_t layer, const int32
   p.num_kv_heads = pool->num_kv_heads;
   p.n_tokens = n_tokens;
   p.row_bytes = pool->head_dim * (pool->dtype == RAG_BF16 ? 2 : 4);
+  p.v_to_f16 = pool->dtype == RAG_BF16 ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   LaunchScope ls(kKindPoolWrite, s);
   cudaError_t e = launch_pool_write(p, n_pages, s);
@@ -705,6 +706,7 @@ rag_status rag_recompute_status(const void* plan, int32_t* counts, void* stream)
   if (bits & kRcErrNoFree) return RAG_ERR_NO_FREE_PAGES;
   if (bits & kDevErrPage) return RAG_ERR_PAGE_OOB;
   if (bits & kDevErrGeometry) return RAG_ERR_GEOMETRY;
+  if (bits & kDevErrRange) return RAG_ERR_RANGE;
   return RAG_OK;
 }
 

@@ -21,8 +21,10 @@
 //                     rows listed by doc position; the B operand (the rows of
 //                     two KV heads of W_K or W_V, one when H_kv is odd) by a
 //                     tiled TMA load; the accumulator lives in TMEM, and the
-//                     epilogue rounds each row to bf16 and stores it into its
-//                     slot of its private page.
+//                     epilogue rounds each row once to the type the pool
+//                     stores it in (K bf16, V fp16: nearest even, V saturated
+//                     beyond 65504 with kDevErrRange raised) and stores it
+//                     into its slot of its private page.
 // Every wait is bounded; a timeout raises a device error instead of hanging.
 // None of these kernels releases its dependents early: they write page tables
 // and pool pages, which the attention kernel reads before its own wait. (Running
@@ -420,18 +422,30 @@ rc_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         if (store) {
           const int ho = nt * hpt + hh;       // output head over K heads then V heads
           const int head = ho % p.num_kv_heads;
-          __nv_bfloat16* pool = ho < p.num_kv_heads ? p.pool_k : p.pool_v;
+          const bool is_v = ho >= p.num_kv_heads;
+          __nv_bfloat16* pool = is_v ? p.pool_v : p.pool_k;
+          bool over = false;
           const int64_t orow = ((int64_t(p.layer) * p.num_pages + page) * p.num_kv_heads + head) * kPage + slot;
           uint4* out = reinterpret_cast<uint4*>(pool + orow * kHeadDim);
 #pragma unroll
           for (int c = 0; c < kRcHead / 8; ++c) {
             uint4 v;
-            v.x = pack_bf16x2(acc[8 * c + 0], acc[8 * c + 1]);
-            v.y = pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]);
-            v.z = pack_bf16x2(acc[8 * c + 4], acc[8 * c + 5]);
-            v.w = pack_bf16x2(acc[8 * c + 6], acc[8 * c + 7]);
+            if (is_v) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) over |= beyond_f16(acc[8 * c + j]);
+              v.x = pack_f16x2_sat(acc[8 * c + 0], acc[8 * c + 1]);
+              v.y = pack_f16x2_sat(acc[8 * c + 2], acc[8 * c + 3]);
+              v.z = pack_f16x2_sat(acc[8 * c + 4], acc[8 * c + 5]);
+              v.w = pack_f16x2_sat(acc[8 * c + 6], acc[8 * c + 7]);
+            } else {
+              v.x = pack_bf16x2(acc[8 * c + 0], acc[8 * c + 1]);
+              v.y = pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]);
+              v.z = pack_bf16x2(acc[8 * c + 4], acc[8 * c + 5]);
+              v.w = pack_bf16x2(acc[8 * c + 6], acc[8 * c + 7]);
+            }
             out[c] = v;
           }
+          if (over) atomicOr(err, kDevErrRange);
         }
       }
     }

@@ -124,14 +124,19 @@ def _check(status: int, where: str):
 # --------------------------------------------------------------------------- pool
 
 class KVPool:
-    """The paged pool [layers][pages][kv_heads][16][head_dim] for K and V."""
+    """The paged pool [layers][pages][kv_heads][16][head_dim] for K and V. A
+    bf16 cache keeps K in bf16 and V in fp16 (the type V enters the product
+    with the attention weights in; rag_kv_pool_write and the decode and
+    recompute kernels store it so)."""
 
     def __init__(self, num_layers, num_pages, num_kv_heads, head_dim, dtype=torch.bfloat16, device="cuda",
                  k=None, v=None):
         shape = (num_layers, num_pages, num_kv_heads, PAGE_SIZE, head_dim)
+        v_dtype = torch.float16 if dtype == torch.bfloat16 else dtype
         self.k = torch.zeros(shape, dtype=dtype, device=device) if k is None else k
-        self.v = torch.zeros(shape, dtype=dtype, device=device) if v is None else v
+        self.v = torch.zeros(shape, dtype=v_dtype, device=device) if v is None else v
         assert tuple(self.k.shape) == shape and tuple(self.v.shape) == shape
+        assert self.k.dtype == dtype and self.v.dtype == v_dtype
         self.c = RagKVPool(self.k.data_ptr(), self.v.data_ptr(), num_layers, num_pages, num_kv_heads, PAGE_SIZE,
                            head_dim, RAG_BF16 if dtype == torch.bfloat16 else RAG_F32)
 

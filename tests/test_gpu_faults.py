@@ -118,23 +118,39 @@ def test_chunk_with_one_page_too_few_is_reported():
     check_other_requests(case, out, ref, skip=bad)
 
 
-@pytest.mark.parametrize("value,flagged", [(65280.0, False), (70000.0, True)])
-def test_v_beyond_the_fp16_range_is_reported(value, flagged):
+@pytest.mark.parametrize("value,flagged", [(65280.0, False), (70000.0, True), (float("inf"), True)])
+def test_v_beyond_the_fp16_range_is_reported_by_the_pool_write(value, flagged):
+    """A bf16 pool keeps V in fp16: 65,280 is exact there; 70,000 and inf
+    saturate to 65,504 and the write reports RAG_ERR_RANGE's bit. The oracle
+    stores V the same way, so attention keeps full parity either way."""
     w = scaled(get_workload("llama2_7b_l1"), num_q_heads=4, num_kv_heads=4, chunk_lens=(200, 77), q_len=20)
     case = DeviceCase(w, layers=[0])
     inp = case.inputs[0]
     inp.chunk_v[0][3, 1, 5] = value                  # one V value of chunk 0 (also the oracle's input)
     pages = case.lay.chunk_pages[0].to(torch.int32).cuda()
-    rag_kv_pool_write(case.pool, 0, pages, inp.chunk_k[0].cuda(), inp.chunk_v[0].cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rag_kv_pool_write(case.pool, 0, pages, inp.chunk_k[0].cuda(), inp.chunk_v[0].cuda(), device_err=err)
     torch.cuda.synchronize()
-    if not flagged:
-        check_layer(case, 0, with_impact=True)       # 65,280 is exact in fp16: full parity, no report
-        return
-    q, kq, vq = case.dev_inputs[0]
-    case.engine.attend(0, q, kq, vq, with_impact=True)
-    torch.cuda.synchronize()
+    assert int(err.item()) == (8 if flagged else 0)
+    stored = case.pool.v[0].float()
+    assert stored.abs().max().item() <= 65504.0
+    check_layer(case, 0, with_impact=True)
+
+
+def test_v_q_beyond_the_fp16_range_is_reported_by_the_attention():
+    """The query block's own V_q enters the product as fp16 too: a value of
+    70,000 is saturated and the call reports RAG_ERR_RANGE; the rest of the
+    output keeps parity with the oracle, which saturates it the same way."""
+    w = scaled(get_workload("llama2_7b_l1"), num_q_heads=4, num_kv_heads=4, chunk_lens=(200, 77), q_len=20)
+    case = DeviceCase(w, layers=[0])
+    inp = case.inputs[0]
+    inp.vq[7, 2, 100] = 70000.0
+    case.dev_inputs[0] = (inp.q.cuda(), inp.kq.cuda(), inp.vq.cuda())
+    out = case.run_layer(0, with_impact=True)
+    ref = case.oracle(0, True)
     st, bits = case.engine.device_error()
     assert st == RAG_ERR_RANGE and bits == 8, (st, bits)
+    assert_o_close(out["o"], ref.o, w.dtype)
 
 
 def test_bounded_wait_gives_up_and_reports_a_timeout():

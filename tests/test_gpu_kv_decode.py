@@ -27,7 +27,7 @@ def build(w, bits, layer=0):
     return lay, encs
 
 
-def run(w, bits, layers=(0, 1)):
+def run(w, bits, layers=(0, 1), tweak=None):
     lay, _ = build(w, bits)
     L = max(layers) + 1
     pool = KVPool(L, lay.num_pages, w.num_kv_heads, w.head_dim, device="cuda")
@@ -38,6 +38,8 @@ def run(w, bits, layers=(0, 1)):
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     for layer in layers:
         _, encs = build(w, bits, layer)
+        if tweak:
+            tweak(encs)
         n = [lay.chunk_len[c] for c in range(len(encs))]
         tok_off = torch.tensor(np.cumsum([0] + n), dtype=torch.int32, device="cuda")
         page_off = torch.tensor(np.cumsum([0] + [len(p) for p in lay.chunk_pages]), dtype=torch.int32, device="cuda")
@@ -71,6 +73,17 @@ def test_decode_is_bit_exact(name, bits):
     got_k, got_v, ref_k, ref_v, err = run(cases()[name], bits)
     assert err == 0
     assert np.array_equal(got_k, ref_k) and np.array_equal(got_v, ref_v)
+
+
+def test_v_beyond_the_fp16_range_is_saturated_and_reported():
+    """V is stored as fp16: a channel whose decoded values reach 70,000 is
+    saturated to 65,504 (the oracle stores the same bits) and bit 8 is set."""
+    def tweak(encs):
+        encs[1].offset_v[0, 3] = 70000.0
+    got_k, got_v, ref_k, ref_v, err = run(cases()["ragged"], 8, layers=(0,), tweak=tweak)
+    assert err == 8
+    assert np.array_equal(got_k, ref_k) and np.array_equal(got_v, ref_v)
+    assert (got_v == 0x7BFF).any()
 
 
 def test_page_outside_the_pool_is_skipped_and_reported():

@@ -1,7 +1,7 @@
 """Parity of the CUDA path (through the C ABI) with the fp64 oracle.
 
 Sizes span several 128-key tiles, several 128-row tiles, ragged chunk tails,
-several requests, GQA groups of 1 to 8, split and unsplit key ranges, and the
+several requests (up to 130), GQA groups of 1 to 8, split and unsplit key ranges, and the
 edge cases of the method (one query token, one-token chunks, a request with
 no query tokens, repeated chunks). The full-size workloads run in the launch
 configuration the benchmark times.
@@ -44,6 +44,10 @@ def small_cases():
         "one_query_token": scaled(l2, num_q_heads=8, num_kv_heads=8, chunk_lens=(1, 15, 16, 17, 129), q_len=1),
         "query_longer_than_tile": scaled(l3, num_layers=1, num_q_heads=4, num_kv_heads=2, chunk_lens=(60,),
                                          q_len=300),
+        # over 117 requests: the attention kernel's V tiles are double- rather
+        # than triple-buffered (the request table takes the shared memory)
+        "many_requests": scaled(b16, num_q_heads=8, num_kv_heads=2, n_requests=130, n_pool_chunks=40,
+                                chunk_len_range=(1, 300), chunks_per_req=(1, 3), q_range=(1, 40)),
     }
 
 

@@ -91,16 +91,17 @@ def run_case(w, sel, spare, layers=(0,), by_selection=False, free_order=None):
     return case, ref_plan, page_out.cpu().numpy(), st, counts, results
 
 
-def assert_pool_matches(ref_plan, ref_bits, got_bits):
-    """Bit-exact everywhere except the recomputed slots, which are within one bf16 step."""
+def assert_pool_matches(ref_plan, ref_bits, got_bits, decode):
+    """Bit-exact everywhere except the recomputed slots, which are within one
+    bf16 step (decode: the stored format's values, bf16 for K, fp16 for V)."""
     sel = np.zeros(ref_bits.shape[:1] + ref_bits.shape[2:3], dtype=bool)   # [pages, slots]
     for page, slot in zip(ref_plan.dst_page, ref_plan.dst_slot):
         sel[page, slot] = True
     keep = ~sel
     assert np.array_equal(ref_bits.transpose(0, 2, 1, 3)[keep], got_bits.transpose(0, 2, 1, 3)[keep])
     if sel.any():
-        r = orc_rc.bits_to_f64(ref_bits.transpose(0, 2, 1, 3)[sel])
-        g = orc_rc.bits_to_f64(got_bits.transpose(0, 2, 1, 3)[sel])
+        r = decode(ref_bits.transpose(0, 2, 1, 3)[sel])
+        g = decode(got_bits.transpose(0, 2, 1, 3)[sel])
         err = np.abs(g - r)
         bound = ATOL + RTOL * np.abs(r)
         assert (err <= bound).all(), f"recomputed rows: worst ratio {(err / bound).max():.3g}"
@@ -121,8 +122,8 @@ def test_recompute_matches_oracle(name, by_selection):
     assert np.array_equal(page_out, ref_plan.new_page_ids)
     assert cnt == (sum(len(s) for s in sel), len(ref_plan.cow_src), ref_plan.n_needed)
     for layer, rk, rv, gk, gv in results:
-        assert_pool_matches(ref_plan, rk, gk)
-        assert_pool_matches(ref_plan, rv, gv)
+        assert_pool_matches(ref_plan, rk, gk, orc.bits_to_f64)
+        assert_pool_matches(ref_plan, rv, gv, orc.f16_bits_to_f64)
 
 
 def test_private_pages_come_from_the_free_list_in_reference_order():
@@ -136,8 +137,8 @@ def test_private_pages_come_from_the_free_list_in_reference_order():
     assert st == 0
     assert np.array_equal(page_out, ref_plan.new_page_ids)
     for layer, rk, rv, gk, gv in results:
-        assert_pool_matches(ref_plan, rk, gk)
-        assert_pool_matches(ref_plan, rv, gv)
+        assert_pool_matches(ref_plan, rk, gk, orc.bits_to_f64)
+        assert_pool_matches(ref_plan, rv, gv, orc.f16_bits_to_f64)
 
 
 def test_too_few_free_pages_leaves_everything_unchanged():
@@ -178,7 +179,8 @@ def test_attention_after_recompute_uses_the_private_pages():
     # oracle attention over its own recomputed pool
     _, rk, rv, _, _ = results[0]
     inp = case.inputs[0]
-    q_all, kq_all, vq_all = orc.to_f64(inp.q), orc.to_f64(inp.kq), orc.to_f64(inp.vq)
+    q_all, kq_all = orc.to_f64(inp.q), orc.to_f64(inp.kq)
+    vq_all = orc.v_values(orc.v_operand_bits(orc.to_bits(inp.vq)))
     o_ref = np.zeros_like(got)
     q0 = 0
     for b, cs in enumerate(lay.req_chunks):
@@ -188,7 +190,7 @@ def test_attention_after_recompute_uses_the_private_pages():
             p0, p1 = int(lay.chunk_page_off[e]), int(lay.chunk_page_off[e + 1])
             chunks.append((ref_plan.new_page_ids[p0:p1], int(lay.chunk_doc_off[e + 1] - lay.chunk_doc_off[e])))
         kd = orc.bits_to_f64(orc.gather(rk[None], 0, chunks))
-        vd = orc.bits_to_f64(orc.gather(rv[None], 0, chunks))
+        vd = orc.v_values(orc.gather(rv[None], 0, chunks))
         kcat = np.concatenate([kd, kq_all[q0:q0 + ql]])
         vcat = np.concatenate([vd, vq_all[q0:q0 + ql]])
         o, _, _, _, _ = orc.attend_request(q_all[q0:q0 + ql], kcat, vcat, kd.shape[0], 1 / np.sqrt(w.head_dim),

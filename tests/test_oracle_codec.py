@@ -3,6 +3,8 @@ it: the quantization error bound of uniform b-bit codes, exact extremes and
 constant channels, a hand-packed 4-bit byte, and the page placement of the
 pool write. A mutation test swaps the nibble order and checks a pin fails."""
 
+import struct
+
 import numpy as np
 import pytest
 import torch
@@ -66,6 +68,13 @@ def test_decode_places_tokens_like_the_pool_write():
     assert np.array_equal(pk, ref)
     # pages the chunk does not own are untouched
     assert np.all(pk[0, [0, 2, 4]] == 0xFFFF)
+    # V: the fp32 value rounded once to binary16 (Python's struct packing)
+    v32 = codec.dequantize_f32(codec.unpack(enc.codes_v, 8), enc.scale_v[None], enc.offset_v[None])
+    want_v = np.frombuffer(struct.pack(f"<{v32.size}e", *v32.astype(np.float64).ravel().tolist()),
+                           dtype=np.uint16).reshape(v32.shape)
+    ref_v = np.full_like(pv, 0xFFFF)
+    orc.pool_write(ref_v, 0, pages, want_v)
+    assert np.array_equal(pv, ref_v)
 
 
 def test_mutation_nibble_order_is_caught(monkeypatch):
