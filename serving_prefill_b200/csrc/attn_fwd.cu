@@ -24,10 +24,10 @@
 // PV runs in fp16 (P and V): P keeps 3 more mantissa bits than bf16, and the
 // pool of a bf16 cache stores V as fp16 already, so doc V tiles go from TMA
 // to the tensor core untouched.
-// kPolyPairsOf8 can move a share of the exponentials onto the FMA pipe
-// (exp2_poly2); measured on B200 this pass runs fastest with all of them on
-// MUFU. Every wait is bounded; a timeout raises a device error instead of
-// hanging.
+// Every exponential runs on MUFU: moving a share of them onto the FMA pipe
+// as a polynomial measured slower on B200 (the softmax warps are bound by
+// their issue rate, not by MUFU). Every wait is bounded; a timeout raises a
+// device error instead of hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -44,7 +44,6 @@ constexpr int kTileBytes = kBN * kHeadDim * 2;   // one K, V or Q tile, 16-bit
 constexpr int kHalfBytes = kTileBytes / 2;       // 64 columns of d
 constexpr int kFwdThreads = 384;                 // 8 softmax + K + V + MMA + convert warps
 constexpr float kRescaleThreshold = 8.0f;        // log2 units: rescale O when the max grows by > 2^8
-constexpr int kPolyPairsOf8 = 0;                 // of every 8 column pairs, this many use the FMA-pipe exp2
 
 // TMEM columns: S_i (P_i aliased over its first 64 columns), O_i
 __host__ __device__ constexpr uint32_t col_s(int qt) { return 128u * qt; }
@@ -392,12 +391,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float2 y = ffma2(make_float2(x[64 * h + 2 * j], x[64 * h + 2 * j + 1]), sc2, nm2);
-            float2 e;
-            if ((j & 7) < kPolyPairsOf8) {
-              e = exp2_poly2(y);
-            } else {
-              e = make_float2(ex2(y.x), ex2(y.y));
-            }
+            const float2 e = make_float2(ex2(y.x), ex2(y.y));
             ls[j & 3] = fadd2(ls[j & 3], e);
             pk[j] = pack_f16x2(e.x, e.y);
           }

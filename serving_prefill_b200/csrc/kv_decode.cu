@@ -24,7 +24,73 @@ namespace rag {
 
 constexpr int kDecThreads = 256;
 
-__global__ void __launch_bounds__(kDecThreads, 4) kv_decode_kernel(const KvDecodeParams p) {
+// 8 channels of one KV head for the 16 slots of a page: codes -> fp32 value
+// fma(code, scale, offset) -> the stored type, rounded once (K: bf16; V:
+// fp16, saturated). A decoded value is linear in its code and rounding is
+// monotonic, so a group whose two end values (code 0 and code 2^b - 1) are
+// within the fp16 range has no V value to check one by one (a nan scale or
+// offset fails that test).
+template <bool kV>
+__device__ __forceinline__ void decode_unit(const KvDecodeParams& p, const uint8_t* codes, int64_t token_stride,
+                                            int grp, int n_valid, const float* scale_p, const float* offset_p,
+                                            uint4* out, bool& over) {
+  const float4 s0 = __ldg(reinterpret_cast<const float4*>(scale_p));
+  const float4 s1 = __ldg(reinterpret_cast<const float4*>(scale_p) + 1);
+  const float4 o0 = __ldg(reinterpret_cast<const float4*>(offset_p));
+  const float4 o1 = __ldg(reinterpret_cast<const float4*>(offset_p) + 1);
+  bool check = false;
+  if (kV) {
+    const float top = float((1 << p.bits) - 1);
+    check = beyond_f16(o0.x) || beyond_f16(o0.y) || beyond_f16(o0.z) || beyond_f16(o0.w) ||
+            beyond_f16(o1.x) || beyond_f16(o1.y) || beyond_f16(o1.z) || beyond_f16(o1.w) ||
+            beyond_f16(__fmaf_rn(top, s0.x, o0.x)) || beyond_f16(__fmaf_rn(top, s0.y, o0.y)) ||
+            beyond_f16(__fmaf_rn(top, s0.z, o0.z)) || beyond_f16(__fmaf_rn(top, s0.w, o0.w)) ||
+            beyond_f16(__fmaf_rn(top, s1.x, o1.x)) || beyond_f16(__fmaf_rn(top, s1.y, o1.y)) ||
+            beyond_f16(__fmaf_rn(top, s1.z, o1.z)) || beyond_f16(__fmaf_rn(top, s1.w, o1.w));
+  }
+  uint2 cw[kPage];
+#pragma unroll
+  for (int slot = 0; slot < kPage; ++slot) {
+    cw[slot] = make_uint2(0u, 0u);
+    if (slot >= n_valid) continue;
+    const uint8_t* cs = codes + slot * token_stride;
+    if (p.bits == 8) cw[slot] = __ldg(reinterpret_cast<const uint2*>(cs + grp * 8));
+    else cw[slot].x = __ldg(reinterpret_cast<const uint32_t*>(cs + grp * 4));
+  }
+#pragma unroll
+  for (int slot = 0; slot < kPage; ++slot) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);   // slots past the chunk's end are zeroed
+    if (slot < n_valid) {
+      float q[8];
+      if (p.bits == 8) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          q[i] = float((cw[slot].x >> (8 * i)) & 0xffu);
+          q[4 + i] = float((cw[slot].y >> (8 * i)) & 0xffu);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = float((cw[slot].x >> (4 * i)) & 0xfu);
+      }
+      const float y0 = __fmaf_rn(q[0], s0.x, o0.x), y1 = __fmaf_rn(q[1], s0.y, o0.y);
+      const float y2 = __fmaf_rn(q[2], s0.z, o0.z), y3 = __fmaf_rn(q[3], s0.w, o0.w);
+      const float y4 = __fmaf_rn(q[4], s1.x, o1.x), y5 = __fmaf_rn(q[5], s1.y, o1.y);
+      const float y6 = __fmaf_rn(q[6], s1.z, o1.z), y7 = __fmaf_rn(q[7], s1.w, o1.w);
+      if (kV) {
+        if (check)
+          over |= beyond_f16(y0) || beyond_f16(y1) || beyond_f16(y2) || beyond_f16(y3) || beyond_f16(y4) ||
+                  beyond_f16(y5) || beyond_f16(y6) || beyond_f16(y7);
+        v = make_uint4(pack_f16x2_sat(y0, y1), pack_f16x2_sat(y2, y3), pack_f16x2_sat(y4, y5),
+                       pack_f16x2_sat(y6, y7));
+      } else {
+        v = make_uint4(pack_bf16x2(y0, y1), pack_bf16x2(y2, y3), pack_bf16x2(y4, y5), pack_bf16x2(y6, y7));
+      }
+    }
+    out[slot * (kHeadDim / 8)] = v;
+  }
+}
+
+__global__ void __launch_bounds__(kDecThreads, 3) kv_decode_kernel(const KvDecodeParams p) {
   // no early release: the attention kernel reads pool pages before its own
   // wait, so it must start only once every page written here is complete
   const int gp = blockIdx.x;   // page of the batch
@@ -62,75 +128,12 @@ __global__ void __launch_bounds__(kDecThreads, 4) kv_decode_kernel(const KvDecod
     const int h = (u / (kHeadDim / 8)) % hk;
     const int grp = u % (kHeadDim / 8);                        // channels 8 grp .. 8 grp + 7
     const int64_t so = (int64_t(c) * hk + h) * kHeadDim + grp * 8;
-    const float4* scale = reinterpret_cast<const float4*>((tensor ? p.scale_v : p.scale_k) + so);
-    const float4* offset = reinterpret_cast<const float4*>((tensor ? p.offset_v : p.offset_k) + so);
-    const float4 s0 = __ldg(scale), s1 = __ldg(scale + 1), o0 = __ldg(offset), o1 = __ldg(offset + 1);
-    // A decoded value is linear in its code, and rounding is monotonic, so
-    // its magnitude is at most that of the ends, code 0 and code 2^b - 1: when
-    // both are within the fp16 range, no V value of the group is checked one
-    // by one (a nan scale or offset fails the test).
-    bool v_checked = false;
-    if (tensor) {
-      const float top = float((1 << p.bits) - 1);
-      const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      const float of[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v_checked = v_checked || beyond_f16(of[i]) || beyond_f16(__fmaf_rn(top, sc[i], of[i]));
-    }
     const uint8_t* codes = (tensor ? p.codes_v : p.codes_k) + (int64_t(t_first) * hk + h) * code_row;
-    const int64_t token_stride = int64_t(hk) * code_row;
-    uint2 cw[kPage];
-#pragma unroll
-    for (int slot = 0; slot < kPage; ++slot) {
-      cw[slot] = make_uint2(0u, 0u);
-      if (slot >= n_valid) continue;
-      const uint8_t* cs = codes + slot * token_stride;
-      if (p.bits == 8) cw[slot] = __ldg(reinterpret_cast<const uint2*>(cs + grp * 8));
-      else cw[slot].x = __ldg(reinterpret_cast<const uint32_t*>(cs + grp * 4));
-    }
     uint4* out = reinterpret_cast<uint4*>((tensor ? p.pool_v : p.pool_k) + page_base) + h * kPage * (kHeadDim / 8) + grp;
-#pragma unroll
-    for (int slot = 0; slot < kPage; ++slot) {
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);   // slots past the chunk's end are zeroed
-      if (slot < n_valid) {
-        float q[8];
-        if (p.bits == 8) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            q[i] = float((cw[slot].x >> (8 * i)) & 0xffu);
-            q[4 + i] = float((cw[slot].y >> (8 * i)) & 0xffu);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) q[i] = float((cw[slot].x >> (4 * i)) & 0xfu);
-        }
-        float y[8];
-        y[0] = __fmaf_rn(q[0], s0.x, o0.x);
-        y[1] = __fmaf_rn(q[1], s0.y, o0.y);
-        y[2] = __fmaf_rn(q[2], s0.z, o0.z);
-        y[3] = __fmaf_rn(q[3], s0.w, o0.w);
-        y[4] = __fmaf_rn(q[4], s1.x, o1.x);
-        y[5] = __fmaf_rn(q[5], s1.y, o1.y);
-        y[6] = __fmaf_rn(q[6], s1.z, o1.z);
-        y[7] = __fmaf_rn(q[7], s1.w, o1.w);
-        if (tensor) {
-          if (v_checked) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) over |= beyond_f16(y[i]);
-          }
-          v.x = pack_f16x2_sat(y[0], y[1]);
-          v.y = pack_f16x2_sat(y[2], y[3]);
-          v.z = pack_f16x2_sat(y[4], y[5]);
-          v.w = pack_f16x2_sat(y[6], y[7]);
-        } else {
-          v.x = pack_bf16x2(y[0], y[1]);
-          v.y = pack_bf16x2(y[2], y[3]);
-          v.z = pack_bf16x2(y[4], y[5]);
-          v.w = pack_bf16x2(y[6], y[7]);
-        }
-      }
-      out[slot * (kHeadDim / 8)] = v;
-    }
+    if (tensor)
+      decode_unit<true>(p, codes, hk * code_row, grp, n_valid, p.scale_v + so, p.offset_v + so, out, over);
+    else
+      decode_unit<false>(p, codes, hk * code_row, grp, n_valid, p.scale_k + so, p.offset_k + so, out, over);
   }
   if (over && p.err) atomicOr(p.err, kDevErrRange);
 }

@@ -53,30 +53,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Same test, but a thread whose phase is not complete is suspended (for up to
-// `hint_ns`) until it completes, instead of spinning on issue slots that the
-// CTA's math warps need.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
 // Waits for the phase of `bar` with the given parity to complete. Gives up
 // (returns false) when `abort` is raised by another role of the CTA or after
-// limit_ns; the caller then raises the abort flag and leaves its loop.
+// limit_ns; the caller then raises the abort flag and leaves its loop. The
+// try_wait without a time hint measured faster on B200 than one with a hint
+// (the waiting thread resumes sooner once the phase completes).
 __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
                                               uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, 50000u)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > limit_ns) return false;
   }
@@ -84,34 +71,6 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, vo
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
-}
-
-// Non-blocking test of a phase (never suspends the thread).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// mbar_wait for a single issuing thread on the critical path: polls without
-// suspending, so it reacts to the phase completing within a few cycles (a
-// suspended try_wait resumes later). Bounded like mbar_wait.
-__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t k = 1;; ++k) {
-    if (mbar_test_wait(bar, parity)) return true;
-    if ((k & 255u) == 0u) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) return false;
-    }
-  }
 }
 
 // ------------------------------------------------------------------ TMA
@@ -352,38 +311,6 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
   return bits_f2(d);
-}
-
-// 2^x on the FMA pipe: x = n + f with n = round(x), f in [-1/2, 1/2];
-// 2^f by a degree-3 polynomial (minimax for relative error on [-1/2, 1/2],
-// fitted for this library with the Remez exchange; max relative error 7.5e-5),
-// 2^n by adding n to the exponent field. Inputs below -126 are clamped (their
-// result, ~1e-38, is below every fp16/fp32 sum it enters).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float magic = 12582912.0f;            // 1.5 * 2^23: x + magic rounds x to an integer
-  const float t = x + magic;
-  const float f = x - (t - magic);
-  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999280571937561f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// exp2_poly on a pair with packed fp32 arithmetic (same method and constants).
-__device__ __forceinline__ float2 exp2_poly2(float2 y) {
-  y.x = fmaxf(y.x, -126.0f);
-  y.y = fmaxf(y.y, -126.0f);
-  const float2 magic = make_float2(12582912.0f, 12582912.0f);
-  const float2 t = fadd2(y, magic);
-  const float2 rn = fadd2(t, make_float2(-12582912.0f, -12582912.0f));   // round(y)
-  const float2 f = ffma2(rn, make_float2(-1.0f, -1.0f), y);                 // y - round(y)
-  float2 p = ffma2(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
-                   make_float2(0.2426111251115799f, 0.2426111251115799f));
-  p = ffma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-  p = ffma2(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
