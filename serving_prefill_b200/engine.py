@@ -59,37 +59,102 @@ class PrefillEngine:
         return rag_last_device_error(self.ws)
 
 
+def layer_groups(per_layer, group_size, device, fill=True):
+    """Pack per-layer tensors into one pinned host buffer and one device buffer
+    per group of `group_size` consecutive layers (the layout HostStep copies
+    in one piece). per_layer[i] is a tuple of tensors of layer i (host or
+    device, any dtype); each gets a 256-byte aligned slot. Returns
+    (groups, host_views, dev_views): groups as HostStep's in_groups /
+    out_groups take them (host buffer, device buffer, [layer positions]), and
+    per layer the tuples of host and device views. fill copies the tensors'
+    values into the host views."""
+    groups, host_views, dev_views = [], [], []
+    for g0 in range(0, len(per_layer), group_size):
+        idx = list(range(g0, min(g0 + group_size, len(per_layer))))
+        offs, at = [], 0
+        for i in idx:
+            row = []
+            for t in per_layer[i]:
+                row.append(at)
+                at += (t.numel() * t.element_size() + 255) // 256 * 256
+            offs.append(row)
+        host = torch.empty(max(at, 256), dtype=torch.uint8).pin_memory()
+        dev = torch.empty(max(at, 256), dtype=torch.uint8, device=device)
+        for i, row in zip(idx, offs):
+            hv, dv = [], []
+            for t, o in zip(per_layer[i], row):
+                nb = t.numel() * t.element_size()
+                h = host[o:o + nb].view(t.dtype).view(t.shape)
+                if fill:
+                    h.copy_(t)
+                hv.append(h)
+                dv.append(dev[o:o + nb].view(t.dtype).view(t.shape))
+            host_views.append(tuple(hv))
+            dev_views.append(tuple(dv))
+        groups.append((host, dev, idx))
+    return groups, host_views, dev_views
+
+
 class HostStep:
     """A whole step from pinned host buffers to pinned host buffers.
 
     The batch descriptors and every layer's q, kq, vq travel host -> device on
     a copy stream, each layer's O travels back on a second one, and the
-    kernels run on the caller's current stream; events order them, so layer
-    l + 1's inputs arrive, and layer l - 1's output leaves, while layer l
+    kernels run on the caller's current stream; events order them, so later
+    layers' inputs arrive, and earlier layers' outputs leave, while a layer
     computes (and the next step's copies start as soon as the buffers they
     overwrite are free). Every step of the method still runs in the library's
-    kernels; this class only schedules the copies around them.
+    kernels; this class only schedules the copies around them. A step's host
+    outputs are complete once host_ready() (an event on the output copy
+    stream) has completed; the next step does not wait for them, only for the
+    device buffers it reuses.
+
+    Copies go either per tensor (host_in[i] = (q, kq, vq), host_out[i]) or, with
+    in_groups / out_groups, per group of consecutive layers: a group is
+    (host buffer, device buffer, [layer positions]) whose layers' device q, kq,
+    vq (or O) are views of the device buffer laid out like the host buffer, so
+    the group moves in one copy and the kernels of its layers follow one
+    another with no event wait between them.
     """
 
     def __init__(self, engine: "PrefillEngine", layers_dev, outs_dev, host_in, host_out, impact_layer,
-                 host_topk=None, batch_host=None):
+                 host_topk=None, batch_host=None, in_groups=None, out_groups=None):
         self.eng = engine
         self.layers_dev = layers_dev        # [(layer, q, kq, vq)] device buffers
         self.outs_dev = outs_dev            # per layer device O
-        self.host_in = host_in              # per layer (q, kq, vq) pinned host tensors
-        self.host_out = host_out            # per layer pinned host O
         self.impact_layer = impact_layer
         self.host_topk = host_topk
         self.batch_host = batch_host        # pinned host copies of the batch descriptor arrays, or None
+        n = len(layers_dev)
+        if in_groups is None:
+            in_groups = [(host_in[i], layers_dev[i][1:], [i]) for i in range(n)]
+        if out_groups is None:
+            out_groups = [(host_out[i], outs_dev[i], [i]) for i in range(n)]
+        for groups in (in_groups, out_groups):
+            order = [i for _, _, idx in groups for i in idx]
+            assert order == list(range(n)), "groups must cover the layers in order"
+        self.in_groups, self.out_groups = in_groups, out_groups
+        self.in_first = {idx[0]: g for g, (_, _, idx) in enumerate(in_groups)}
+        self.out_first = {idx[0]: g for g, (_, _, idx) in enumerate(out_groups)}
+        self.out_last = {idx[-1]: g for g, (_, _, idx) in enumerate(out_groups)}
         self.s_in = torch.cuda.Stream()
         self.s_out = torch.cuda.Stream()
-        n = len(layers_dev)
-        self.ev_in = [torch.cuda.Event() for _ in range(n)]
-        self.ev_done = [torch.cuda.Event() for _ in range(n)]
-        self.ev_out = [torch.cuda.Event() for _ in range(n)]
+        self.ev_in = [torch.cuda.Event() for _ in in_groups]
+        self.ev_used = [torch.cuda.Event() for _ in in_groups]     # the group's inputs are read
+        self.ev_done = [torch.cuda.Event() for _ in out_groups]    # the group's outputs are written
+        self.ev_out = [torch.cuda.Event() for _ in out_groups]     # the group's outputs have left
         self.ev_desc = torch.cuda.Event()
         self.ev_step = torch.cuda.Event()
+        self.ev_host = torch.cuda.Event()
         self.started = False
+
+    @staticmethod
+    def _copy(dst, src):
+        if isinstance(src, (tuple, list)):
+            for d, s_ in zip(dst, src):
+                d.copy_(s_, non_blocking=True)
+        else:
+            dst.copy_(src, non_blocking=True)
 
     def __call__(self):
         cur = torch.cuda.current_stream()
@@ -104,32 +169,43 @@ class HostStep:
                     if t.numel():
                         dt[: t.numel()].copy_(t, non_blocking=True)
                 self.ev_desc.record(self.s_in)
-            for i in range(n):
+            for g, (host, dev, _) in enumerate(self.in_groups):
                 if self.started:
-                    self.s_in.wait_event(self.ev_done[i])  # the previous step's layer i has read them
-                _, q, kq, vq = self.layers_dev[i]
-                hq, hkq, hvq = self.host_in[i]
-                q.copy_(hq, non_blocking=True)
-                kq.copy_(hkq, non_blocking=True)
-                vq.copy_(hvq, non_blocking=True)
-                self.ev_in[i].record(self.s_in)
+                    self.s_in.wait_event(self.ev_used[g])  # the previous step has read this group
+                self._copy(dev, host)
+                self.ev_in[g].record(self.s_in)
         if self.batch_host is not None:
             cur.wait_event(self.ev_desc)
+        in_last = {idx[-1]: g for g, (_, _, idx) in enumerate(self.in_groups)}
         for i in range(n):
             layer, q, kq, vq = self.layers_dev[i]
-            cur.wait_event(self.ev_in[i])
-            if self.started:
-                cur.wait_event(self.ev_out[i])             # the previous step's O of this layer has left
+            if i in self.in_first:
+                cur.wait_event(self.ev_in[self.in_first[i]])
+            if self.started and i in self.out_first:
+                cur.wait_event(self.ev_out[self.out_first[i]])   # the previous step's O of the group has left
             self.eng.attend(layer, q, kq, vq, with_impact=(layer == self.impact_layer), o=self.outs_dev[i])
-            self.ev_done[i].record(cur)
-            with torch.cuda.stream(self.s_out):
-                self.s_out.wait_event(self.ev_done[i])
-                self.host_out[i].copy_(self.outs_dev[i], non_blocking=True)
-                self.ev_out[i].record(self.s_out)
+            if i in in_last:
+                self.ev_used[in_last[i]].record(cur)
+            if i in self.out_last:
+                g = self.out_last[i]
+                self.ev_done[g].record(cur)
+                host, dev, _ = self.out_groups[g]
+                with torch.cuda.stream(self.s_out):
+                    self.s_out.wait_event(self.ev_done[g])
+                    self._copy(host, dev)
+                    self.ev_out[g].record(self.s_out)
         if self.impact_layer is not None:
+            if self.started:
+                cur.wait_event(self.ev_host)   # the previous step's top-k has left
             self.eng.select()
-            if self.host_topk is not None:
-                self.host_topk.copy_(self.eng.topk_idx, non_blocking=True)
         self.ev_step.record(cur)
-        cur.wait_stream(self.s_out)                        # the step ends when its last output has left
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(self.ev_step)
+            if self.impact_layer is not None and self.host_topk is not None:
+                self.host_topk.copy_(self.eng.topk_idx, non_blocking=True)
+            self.ev_host.record(self.s_out)
         self.started = True
+
+    def host_ready(self) -> torch.cuda.Event:
+        """Event after the last device -> host copy of the latest step."""
+        return self.ev_host

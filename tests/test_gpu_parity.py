@@ -179,7 +179,7 @@ def test_host_step_matches_the_device_step():
     """The pipelined step from pinned host buffers (copies on their own
     streams, ordered by events) gives the same outputs as the plain step,
     twice in a row."""
-    from serving_prefill_b200.engine import HostStep
+    from serving_prefill_b200.engine import HostStep, layer_groups
     w = CASES["gqa4_rows3"]
     case = DeviceCase(w)
     layers = [(l,) + case.dev_inputs[l] for l in case.layers]
@@ -196,10 +196,16 @@ def test_host_step_matches_the_device_step():
     desc = [t.contiguous().pin_memory() for t in case.batch.host]
     step = HostStep(case.engine, dev_in, dev_out, host_in, host_out, w.impact_layer_index, host_topk=host_topk,
                     batch_host=desc)
-    for _ in range(2):
-        step()
+    # the same step with every layer's inputs, and every layer's O, moved as one group
+    in_groups, _, gdev_in = layer_groups([case.dev_inputs[l] for l in case.layers], len(layers), "cuda")
+    out_groups, gout_host, gout_dev = layer_groups([(o,) for o in outs], len(layers), "cuda", fill=False)
+    gstep = HostStep(case.engine, [(l,) + gdev_in[n] for n, l in enumerate(case.layers)], [v[0] for v in gout_dev],
+                     None, None, w.impact_layer_index, host_topk=host_topk, batch_host=desc, in_groups=in_groups,
+                     out_groups=out_groups)
+    for run, got in [(step, host_out)] * 2 + [(gstep, [v[0] for v in gout_host])] * 2:
+        run()
         torch.cuda.synchronize()
-        for a, b in zip(host_out, want_o):
+        for a, b in zip(got, want_o):
             assert torch.equal(a[: case.batch.total_q], b[: case.batch.total_q].cpu())   # O is run-to-run stable
         # the selection that came back is the one on the device (Impact sums by
         # atomics, so near-ties may order differently from the first run)
