@@ -139,6 +139,7 @@ class HostStep:
         self.out_last = {idx[-1]: g for g, (_, _, idx) in enumerate(out_groups)}
         self.s_in = torch.cuda.Stream()
         self.s_out = torch.cuda.Stream()
+        self.s_desc = torch.cuda.Stream()
         self.ev_in = [torch.cuda.Event() for _ in in_groups]
         self.ev_used = [torch.cuda.Event() for _ in in_groups]     # the group's inputs are read
         self.ev_done = [torch.cuda.Event() for _ in out_groups]    # the group's outputs are written
@@ -159,16 +160,22 @@ class HostStep:
     def __call__(self):
         cur = torch.cuda.current_stream()
         n = len(self.layers_dev)
-        with torch.cuda.stream(self.s_in):
-            # a step's copies begin after everything the caller queued before it
+        if not self.started:
+            # the first step's copies begin after everything the caller queued
+            # before it; later steps are ordered by the events below alone
             self.s_in.wait_stream(cur)
-            if self.batch_host is not None:
+            self.s_desc.wait_stream(cur)
+        if self.batch_host is not None:
+            # the batch descriptors on their own stream: they wait for the
+            # previous step's end, the layers' inputs only for their buffers
+            with torch.cuda.stream(self.s_desc):
                 if self.started:
-                    self.s_in.wait_event(self.ev_step)     # the previous step no longer reads them
+                    self.s_desc.wait_event(self.ev_step)   # the previous step no longer reads them
                 for t, dt in zip(self.batch_host, self.eng.batch.dev):
                     if t.numel():
                         dt[: t.numel()].copy_(t, non_blocking=True)
-                self.ev_desc.record(self.s_in)
+                self.ev_desc.record(self.s_desc)
+        with torch.cuda.stream(self.s_in):
             for g, (host, dev, _) in enumerate(self.in_groups):
                 if self.started:
                     self.s_in.wait_event(self.ev_used[g])  # the previous step has read this group
