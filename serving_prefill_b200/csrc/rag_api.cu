@@ -101,24 +101,68 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 tensor with rank dims (innermost first), 128B swizzle, zero fill
+// Encoded maps are kept per host thread (no lock), keyed by everything the
+// encoding reads, so that a call whose tensors were seen before (the layers
+// of a step, the steps of a serving loop) skips the driver call. A map holds
+// only the address and the geometry, so a key match is an exact reuse.
+struct MapKey {
+  const void* base;
+  int rank;
+  uint64_t dims[3];
+  uint64_t strides[2];
+  uint32_t box[3];
+  bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+constexpr int kMapCache = 128;
+struct MapCache {
+  MapKey key[kMapCache];
+  CUtensorMap map[kMapCache];
+  int n = 0, next = 0;
+};
+
+// bf16 tensor with rank (<= 3) dims (innermost first), 128B swizzle, zero fill
 static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
                      const uint32_t* box) {
+  MapKey k;
+  std::memset(&k, 0, sizeof(k));   // padding too: keys compare as bytes
+  k.base = base;
+  k.rank = rank;
+  for (int i = 0; i < rank; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+    if (i + 1 < rank) k.strides[i] = strides_bytes[i];
+  }
+  thread_local MapCache cache;
+  for (int i = 0; i < cache.n; ++i)
+    if (cache.key[i] == k) {
+      *m = cache.map[i];
+      return true;
+    }
   auto fn = encode_fn();
   if (!fn) return false;
   uint32_t elem_strides[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes, box,
                   elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  const int slot = cache.n < kMapCache ? cache.n++ : (cache.next++ % kMapCache);
+  cache.key[slot] = k;
+  cache.map[slot] = *m;
+  return true;
 }
 
 // ------------------------------------------------------------ helpers
 
 static int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  thread_local int known[kMaxDevices] = {};   // per device, read once per host thread
+  if (known[dev] <= 0) {
+    int n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    known[dev] = n;
+  }
+  return known[dev];
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -136,7 +180,31 @@ struct Plan {
 // Split the key tiles of every (request, kv head, row block) unit so that
 // the work fills the SMs in whole waves. rows_per_unit: 128 (attention) or
 // 256 (impact).
+static Plan plan_split_uncached(const rag_batch& b, int num_kv_heads, int group, int rows_per_unit, int sms);
+
+// plan_split reads only these batch totals and the shape, so its result is
+// kept per host thread for the last few distinct inputs (every layer of a
+// step, every step of a batch reuses one).
 static Plan plan_split(const rag_batch& b, int num_kv_heads, int group, int rows_per_unit, int sms) {
+  struct Key {
+    int32_t v[10];
+  };
+  constexpr int kPlanCache = 8;
+  thread_local Key keys[kPlanCache];
+  thread_local Plan plans[kPlanCache];
+  thread_local int n = 0, next = 0;
+  Key k = {{b.num_requests, b.max_pages, b.max_q, b.total_q, b.num_page_refs, num_kv_heads, group, rows_per_unit,
+            sms, 0}};
+  for (int i = 0; i < n; ++i)
+    if (std::memcmp(&keys[i], &k, sizeof(Key)) == 0) return plans[i];
+  const Plan pl = plan_split_uncached(b, num_kv_heads, group, rows_per_unit, sms);
+  const int slot = n < kPlanCache ? n++ : (next++ % kPlanCache);
+  keys[slot] = k;
+  plans[slot] = pl;
+  return pl;
+}
+
+static Plan plan_split_uncached(const rag_batch& b, int num_kv_heads, int group, int rows_per_unit, int sms) {
   Plan pl;
   const int B = std::max(1, b.num_requests);
   const int tiles_max = cdiv(b.max_pages, kPagesPerTile) + cdiv(b.max_q, kBN);
