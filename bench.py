@@ -389,7 +389,7 @@ def run_e2e(args, w, lay, layer_inputs, rep, device, world):
     d2h = (host_topk.numel() * 4 if w.select else 0) + sum(o[0].numel() * o[0].element_size() for o in host_o)
     steps = max(3, min(args.steps, 50))
     one = HostStep(eng, dev_in, [v[0] for v in out_dev], None, None, w.impact_layer_index, host_topk=host_topk,
-                   batch_host=desc, in_groups=in_groups, out_groups=out_groups)
+                   batch_host=desc, in_groups=in_groups, out_groups=out_groups, depth=2)
     for _ in range(3):
         one()
     torch.cuda.synchronize()
@@ -404,8 +404,8 @@ def run_e2e(args, w, lay, layer_inputs, rep, device, world):
     doc = sum(lay.doc_lens)
     return {"value": whole_job_rate(world, doc, steps, ms), "unit": "doc-KV tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps,
-            "overlap": f"host copies on two copy streams, one copy per {E2E_GROUP} layers each way, "
-                       "ordered against the kernels by events"}
+            "overlap": f"host copies on copy streams, one copy per {E2E_GROUP} layers each way, two device "
+                       "buffer sets alternating between steps, ordered against the kernels by events"}
 
 
 # ----------------------------------------------------------------------------- selective recompute

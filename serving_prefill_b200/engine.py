@@ -99,15 +99,12 @@ class HostStep:
     """A whole step from pinned host buffers to pinned host buffers.
 
     The batch descriptors and every layer's q, kq, vq travel host -> device on
-    a copy stream, each layer's O travels back on a second one, and the
-    kernels run on the caller's current stream; events order them, so later
-    layers' inputs arrive, and earlier layers' outputs leave, while a layer
-    computes (and the next step's copies start as soon as the buffers they
-    overwrite are free). Every step of the method still runs in the library's
-    kernels; this class only schedules the copies around them. A step's host
-    outputs are complete once host_ready() (an event on the output copy
-    stream) has completed; the next step does not wait for them, only for the
-    device buffers it reuses.
+    copy streams, each layer's O travels back on another one, and the kernels
+    run on the caller's current stream; events order them, so later layers'
+    inputs arrive, and earlier layers' outputs leave, while a layer computes.
+    Every step of the method still runs in the library's kernels; this class
+    only schedules the copies around them. A step's host outputs are complete
+    once host_ready() (an event on the output copy stream) has completed.
 
     Copies go either per tensor (host_in[i] = (q, kq, vq), host_out[i]) or, with
     in_groups / out_groups, per group of consecutive layers: a group is
@@ -115,13 +112,19 @@ class HostStep:
     vq (or O) are views of the device buffer laid out like the host buffer, so
     the group moves in one copy and the kernels of its layers follow one
     another with no event wait between them.
+
+    depth = 2 keeps a second set of device inputs, outputs and batch
+    descriptors, and consecutive steps alternate between the two sets: a
+    step's uploads then wait only for the step before the previous one, so
+    they run while the previous step computes. The host buffers are shared by
+    both sets: a caller that rewrites them between steps waits for the copies
+    of the step that read them (host_ready() of that step covers them).
     """
 
     def __init__(self, engine: "PrefillEngine", layers_dev, outs_dev, host_in, host_out, impact_layer,
-                 host_topk=None, batch_host=None, in_groups=None, out_groups=None):
+                 host_topk=None, batch_host=None, in_groups=None, out_groups=None, depth=1):
+        assert depth in (1, 2)
         self.eng = engine
-        self.layers_dev = layers_dev        # [(layer, q, kq, vq)] device buffers
-        self.outs_dev = outs_dev            # per layer device O
         self.impact_layer = impact_layer
         self.host_topk = host_topk
         self.batch_host = batch_host        # pinned host copies of the batch descriptor arrays, or None
@@ -133,21 +136,53 @@ class HostStep:
         for groups in (in_groups, out_groups):
             order = [i for _, _, idx in groups for i in idx]
             assert order == list(range(n)), "groups must cover the layers in order"
-        self.in_groups, self.out_groups = in_groups, out_groups
         self.in_first = {idx[0]: g for g, (_, _, idx) in enumerate(in_groups)}
+        self.in_last = {idx[-1]: g for g, (_, _, idx) in enumerate(in_groups)}
         self.out_first = {idx[0]: g for g, (_, _, idx) in enumerate(out_groups)}
         self.out_last = {idx[-1]: g for g, (_, _, idx) in enumerate(out_groups)}
+        self.sets = [self._new_set(layers_dev, outs_dev, in_groups, out_groups, engine.batch)]
+        if depth == 2:
+            self.sets.append(self._second_set(layers_dev, outs_dev, in_groups, out_groups, engine.batch))
         self.s_in = torch.cuda.Stream()
         self.s_out = torch.cuda.Stream()
         self.s_desc = torch.cuda.Stream()
-        self.ev_in = [torch.cuda.Event() for _ in in_groups]
-        self.ev_used = [torch.cuda.Event() for _ in in_groups]     # the group's inputs are read
-        self.ev_done = [torch.cuda.Event() for _ in out_groups]    # the group's outputs are written
-        self.ev_out = [torch.cuda.Event() for _ in out_groups]     # the group's outputs have left
-        self.ev_desc = torch.cuda.Event()
-        self.ev_step = torch.cuda.Event()
         self.ev_host = torch.cuda.Event()
-        self.started = False
+        self.steps = 0
+
+    @staticmethod
+    def _new_set(layers_dev, outs_dev, in_groups, out_groups, batch):
+        return {"layers": layers_dev, "outs": outs_dev, "in": in_groups, "out": out_groups, "batch": batch,
+                "ev_in": [torch.cuda.Event() for _ in in_groups],
+                "ev_used": [torch.cuda.Event() for _ in in_groups],    # the group's inputs are read
+                "ev_done": [torch.cuda.Event() for _ in out_groups],   # the group's outputs are written
+                "ev_out": [torch.cuda.Event() for _ in out_groups],    # the group's outputs have left
+                "ev_desc": torch.cuda.Event(), "ev_step": torch.cuda.Event(), "used": False}
+
+    @classmethod
+    def _second_set(cls, layers_dev, outs_dev, in_groups, out_groups, batch):
+        """Device buffers like the first set's (views at the same offsets of
+        new group buffers) and a second device copy of the batch descriptors."""
+        def twin(groups, tensors_of):
+            new_groups, remap = [], {}
+            for host, dev, idx in groups:
+                if isinstance(dev, (tuple, list)):
+                    dev2 = tuple(torch.empty_like(t) for t in dev)
+                    for t, t2 in zip(dev, dev2):
+                        remap[t.data_ptr()] = t2
+                else:
+                    dev2 = torch.empty_like(dev)
+                    for i in idx:
+                        for t in tensors_of(i):
+                            off = t.data_ptr() - dev.data_ptr()
+                            nb = t.numel() * t.element_size()
+                            remap[t.data_ptr()] = dev2[off:off + nb].view(t.dtype).view(t.shape)
+                new_groups.append((host, dev2, idx))
+            return new_groups, remap
+        in2, rin = twin(in_groups, lambda i: layers_dev[i][1:])
+        out2, rout = twin(out_groups, lambda i: (outs_dev[i],))
+        layers2 = [(l[0],) + tuple(rin[t.data_ptr()] for t in l[1:]) for l in layers_dev]
+        outs2 = [rout[o.data_ptr()] for o in outs_dev]
+        return cls._new_set(layers2, outs2, in2, out2, Batch(*batch.host, device=batch.dev[0].device))
 
     @staticmethod
     def _copy(dst, src):
@@ -159,59 +194,62 @@ class HostStep:
 
     def __call__(self):
         cur = torch.cuda.current_stream()
-        n = len(self.layers_dev)
-        if not self.started:
+        st = self.sets[self.steps % len(self.sets)]
+        n = len(st["layers"])
+        if self.steps == 0:
             # the first step's copies begin after everything the caller queued
             # before it; later steps are ordered by the events below alone
             self.s_in.wait_stream(cur)
             self.s_desc.wait_stream(cur)
         if self.batch_host is not None:
-            # the batch descriptors on their own stream: they wait for the
-            # previous step's end, the layers' inputs only for their buffers
+            # the batch descriptors on their own stream: they wait for the end
+            # of the last step that used this set, the layers' inputs only for
+            # their buffers
             with torch.cuda.stream(self.s_desc):
-                if self.started:
-                    self.s_desc.wait_event(self.ev_step)   # the previous step no longer reads them
-                for t, dt in zip(self.batch_host, self.eng.batch.dev):
+                if st["used"]:
+                    self.s_desc.wait_event(st["ev_step"])
+                for t, dt in zip(self.batch_host, st["batch"].dev):
                     if t.numel():
                         dt[: t.numel()].copy_(t, non_blocking=True)
-                self.ev_desc.record(self.s_desc)
+                st["ev_desc"].record(self.s_desc)
         with torch.cuda.stream(self.s_in):
-            for g, (host, dev, _) in enumerate(self.in_groups):
-                if self.started:
-                    self.s_in.wait_event(self.ev_used[g])  # the previous step has read this group
+            for g, (host, dev, _) in enumerate(st["in"]):
+                if st["used"]:
+                    self.s_in.wait_event(st["ev_used"][g])   # the last step of this set has read this group
                 self._copy(dev, host)
-                self.ev_in[g].record(self.s_in)
+                st["ev_in"][g].record(self.s_in)
         if self.batch_host is not None:
-            cur.wait_event(self.ev_desc)
-        in_last = {idx[-1]: g for g, (_, _, idx) in enumerate(self.in_groups)}
+            cur.wait_event(st["ev_desc"])
+        self.eng.batch = st["batch"]
         for i in range(n):
-            layer, q, kq, vq = self.layers_dev[i]
+            layer, q, kq, vq = st["layers"][i]
             if i in self.in_first:
-                cur.wait_event(self.ev_in[self.in_first[i]])
-            if self.started and i in self.out_first:
-                cur.wait_event(self.ev_out[self.out_first[i]])   # the previous step's O of the group has left
-            self.eng.attend(layer, q, kq, vq, with_impact=(layer == self.impact_layer), o=self.outs_dev[i])
-            if i in in_last:
-                self.ev_used[in_last[i]].record(cur)
+                cur.wait_event(st["ev_in"][self.in_first[i]])
+            if st["used"] and i in self.out_first:
+                cur.wait_event(st["ev_out"][self.out_first[i]])   # that step's O of the group has left
+            self.eng.attend(layer, q, kq, vq, with_impact=(layer == self.impact_layer), o=st["outs"][i])
+            if i in self.in_last:
+                st["ev_used"][self.in_last[i]].record(cur)
             if i in self.out_last:
                 g = self.out_last[i]
-                self.ev_done[g].record(cur)
-                host, dev, _ = self.out_groups[g]
+                st["ev_done"][g].record(cur)
+                host, dev, _ = st["out"][g]
                 with torch.cuda.stream(self.s_out):
-                    self.s_out.wait_event(self.ev_done[g])
+                    self.s_out.wait_event(st["ev_done"][g])
                     self._copy(host, dev)
-                    self.ev_out[g].record(self.s_out)
+                    st["ev_out"][g].record(self.s_out)
         if self.impact_layer is not None:
-            if self.started:
+            if self.steps > 0:
                 cur.wait_event(self.ev_host)   # the previous step's top-k has left
             self.eng.select()
-        self.ev_step.record(cur)
+        st["ev_step"].record(cur)
         with torch.cuda.stream(self.s_out):
-            self.s_out.wait_event(self.ev_step)
+            self.s_out.wait_event(st["ev_step"])
             if self.impact_layer is not None and self.host_topk is not None:
                 self.host_topk.copy_(self.eng.topk_idx, non_blocking=True)
             self.ev_host.record(self.s_out)
-        self.started = True
+        st["used"] = True
+        self.steps += 1
 
     def host_ready(self) -> torch.cuda.Event:
         """Event after the last device -> host copy of the latest step."""

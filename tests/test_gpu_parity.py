@@ -202,7 +202,12 @@ def test_host_step_matches_the_device_step():
     gstep = HostStep(case.engine, [(l,) + gdev_in[n] for n, l in enumerate(case.layers)], [v[0] for v in gout_dev],
                      None, None, w.impact_layer_index, host_topk=host_topk, batch_host=desc, in_groups=in_groups,
                      out_groups=out_groups)
-    for run, got in [(step, host_out)] * 2 + [(gstep, [v[0] for v in gout_host])] * 2:
+    # and two-deep: consecutive steps alternate between two device buffer sets
+    dstep = HostStep(case.engine, [(l,) + gdev_in[n] for n, l in enumerate(case.layers)], [v[0] for v in gout_dev],
+                     None, None, w.impact_layer_index, host_topk=host_topk, batch_host=desc, in_groups=in_groups,
+                     out_groups=out_groups, depth=2)
+    for run, got in ([(step, host_out)] * 2 + [(gstep, [v[0] for v in gout_host])] * 2 +
+                     [(dstep, [v[0] for v in gout_host])] * 3):
         run()
         torch.cuda.synchronize()
         for a, b in zip(got, want_o):
