@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "rag_prefill.h"
@@ -113,12 +114,15 @@ struct MapKey {
   uint32_t box[3];
   bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
 };
-constexpr int kMapCache = 128;
-struct MapCache {
-  MapKey key[kMapCache];
-  CUtensorMap map[kMapCache];
-  int n = 0, next = 0;
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    const unsigned char* b = reinterpret_cast<const unsigned char*>(&k);
+    uint64_t h = 1469598103934665603ull;   // FNV-1a over the key's bytes
+    for (size_t i = 0; i < sizeof(MapKey); ++i) h = (h ^ b[i]) * 1099511628211ull;
+    return size_t(h);
+  }
 };
+constexpr size_t kMapCacheMax = 4096;   // entries kept per host thread before the cache starts over
 
 // bf16 tensor with rank (<= 3) dims (innermost first), 128B swizzle, zero fill
 static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
@@ -132,12 +136,12 @@ static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
     k.box[i] = box[i];
     if (i + 1 < rank) k.strides[i] = strides_bytes[i];
   }
-  thread_local MapCache cache;
-  for (int i = 0; i < cache.n; ++i)
-    if (cache.key[i] == k) {
-      *m = cache.map[i];
-      return true;
-    }
+  thread_local std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+  const auto hit = cache.find(k);
+  if (hit != cache.end()) {
+    *m = hit->second;
+    return true;
+  }
   auto fn = encode_fn();
   if (!fn) return false;
   uint32_t elem_strides[5] = {1, 1, 1, 1, 1};
@@ -145,9 +149,8 @@ static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
                   elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return false;
-  const int slot = cache.n < kMapCache ? cache.n++ : (cache.next++ % kMapCache);
-  cache.key[slot] = k;
-  cache.map[slot] = *m;
+  if (cache.size() >= kMapCacheMax) cache.clear();
+  cache.emplace(k, *m);
   return true;
 }
 
