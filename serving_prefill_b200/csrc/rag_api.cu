@@ -183,12 +183,14 @@ struct Plan {
 // Split the key tiles of every (request, kv head, row block) unit so that
 // the work fills the SMs in whole waves. rows_per_unit: 128 (attention) or
 // 256 (impact).
-static Plan plan_split_uncached(const rag_batch& b, int num_kv_heads, int group, int rows_per_unit, int sms);
+enum class PlanFor { kAttention, kImpact };
+static Plan plan_split_uncached(const rag_batch& b, int num_kv_heads, int group, int rows_per_unit, int sms,
+                                PlanFor what);
 
 // plan_split reads only these batch totals and the shape, so its result is
 // kept per host thread for the last few distinct inputs (every layer of a
 // step, every step of a batch reuses one).
-static Plan plan_split(const rag_batch& b, int num_kv_heads, int group, int rows_per_unit, int sms) {
+static Plan plan_split(const rag_batch& b, int num_kv_heads, int group, int rows_per_unit, int sms, PlanFor what) {
   struct Key {
     int32_t v[10];
   };
@@ -197,17 +199,18 @@ static Plan plan_split(const rag_batch& b, int num_kv_heads, int group, int rows
   thread_local Plan plans[kPlanCache];
   thread_local int n = 0, next = 0;
   Key k = {{b.num_requests, b.max_pages, b.max_q, b.total_q, b.num_page_refs, num_kv_heads, group, rows_per_unit,
-            sms, 0}};
+            sms, int32_t(what)}};
   for (int i = 0; i < n; ++i)
     if (std::memcmp(&keys[i], &k, sizeof(Key)) == 0) return plans[i];
-  const Plan pl = plan_split_uncached(b, num_kv_heads, group, rows_per_unit, sms);
+  const Plan pl = plan_split_uncached(b, num_kv_heads, group, rows_per_unit, sms, what);
   const int slot = n < kPlanCache ? n++ : (next++ % kPlanCache);
   keys[slot] = k;
   plans[slot] = pl;
   return pl;
 }
 
-static Plan plan_split_uncached(const rag_batch& b, int num_kv_heads, int group, int rows_per_unit, int sms) {
+static Plan plan_split_uncached(const rag_batch& b, int num_kv_heads, int group, int rows_per_unit, int sms,
+                                PlanFor what) {
   Plan pl;
   const int B = std::max(1, b.num_requests);
   const int tiles_max = cdiv(b.max_pages, kPagesPerTile) + cdiv(b.max_q, kBN);
@@ -223,7 +226,13 @@ static Plan plan_split_uncached(const rag_batch& b, int num_kv_heads, int group,
   // ceil(items / sms) of them. Several requests: items differ in length and
   // are dealt out round-robin, so the estimate is the list-scheduling bound,
   // the average load per SM plus one longest item.
-  constexpr double kItemOverheadTiles = 2.0;   // measured: 2 beats 3 by 5.5% on 16 batched requests, equal elsewhere
+  // Measured: 2 beats 3 by 5.5 % on 16 batched requests, equal elsewhere; an
+  // attention unit of one Q tile (at most 128 rows: decode steps, one query
+  // head per KV head) runs its tiles faster (two S buffers, one softmax
+  // warpgroup), so its fixed cost is more tiles' worth: 4 beats 2 by 15 % on
+  // the 16-request decode step.
+  const bool one_q_tile = what == PlanFor::kAttention && avg_q * group <= kBM;
+  const double kItemOverheadTiles = one_q_tile ? 4.0 : 2.0;
   const double total_tiles = units * tiles_avg;
   double best = 1e300;
   int best_ts = std::max(tiles_max, 1);
@@ -297,7 +306,7 @@ static BatchDev to_dev(const rag_batch& b) {
 
 static size_t workspace_bytes_for(const rag_kv_pool& pool, const rag_batch& b, int num_q_heads) {
   const int G = num_q_heads / pool.num_kv_heads;
-  const Plan pf = plan_split(b, pool.num_kv_heads, G, kFwdRows, num_sms());
+  const Plan pf = plan_split(b, pool.num_kv_heads, G, kFwdRows, num_sms(), PlanFor::kAttention);
   const bool bf16 = pool.dtype == RAG_BF16;
   return ws_layout(b.total_q, num_q_heads, bf16 ? pf.max_items : 0, bf16 ? b.num_chunks : 0).total;
 }
@@ -455,7 +464,7 @@ static rag_status fused_prefill(const rag_kv_pool* pool, int32_t layer, const ra
   // ---- bf16 tensor-core path
   if (kBM % G != 0) return RAG_ERR_UNSUPPORTED;
   const int sms = num_sms();
-  const Plan pf = plan_split(b, pool->num_kv_heads, G, kFwdRows, sms);
+  const Plan pf = plan_split(b, pool->num_kv_heads, G, kFwdRows, sms, PlanFor::kAttention);
   const WsLayout wl = ws_layout(b.total_q, num_q_heads, pf.max_items, b.num_chunks);
   const int H_kv = pool->num_kv_heads;
   const uint64_t pool_rows = uint64_t(pool->num_layers) * pool->num_pages * H_kv * kPage;
@@ -537,7 +546,7 @@ static rag_status fused_prefill(const rag_kv_pool* pool, int32_t layer, const ra
     if (e != cudaSuccess) return RAG_ERR_CUDA;
   }
   if (impact) {
-    const Plan pi = plan_split(b, H_kv, G, kImpactRows, sms);
+    const Plan pi = plan_split(b, H_kv, G, kImpactRows, sms, PlanFor::kImpact);
     ImpactParams ip;
     ip.batch = fp.batch;
     ip.num_pages = pool->num_pages;
