@@ -242,7 +242,9 @@ cudaError_t launch_rc_gemm(const CUtensorMap&, const CUtensorMap&, const CUtenso
 
 cudaError_t launch_attn_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                             const CUtensorMap&, const FwdParams&, int, cudaStream_t);
-cudaError_t launch_attn_combine(const CombineParams&, int, int, cudaStream_t);
+// max_block_rows: rows of the longest 256-row block of any request (max_q * G, at most 256)
+cudaError_t launch_attn_combine(const CombineParams&, int max_rb, int max_block_rows, int num_requests,
+                                cudaStream_t);
 cudaError_t launch_rope_table(const BatchDev&, double base, float2* table, cudaStream_t);
 cudaError_t launch_impact(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const ImpactParams&, int,
                           cudaStream_t);

@@ -541,7 +541,8 @@ static rag_status fused_prefill(const rag_kv_pool* pool, int32_t layer, const ra
     cp.row_m2 = row_m2;
     cp.row_il = row_il;
     LaunchScope ls(kKindCombine, s);
-    cudaError_t e = launch_attn_combine(cp, pf.max_units_rt, b.num_requests, s);
+    const int64_t block_rows = std::min<int64_t>(kFwdRows, int64_t(b.max_q) * G);
+    cudaError_t e = launch_attn_combine(cp, pf.max_units_rt, int(block_rows), b.num_requests, s);
     ls.done(e);
     if (e != cudaSuccess) return RAG_ERR_CUDA;
   }
