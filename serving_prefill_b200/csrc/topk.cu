@@ -16,6 +16,14 @@
 // d1's candidates together exceed the 20,480 that shared memory stages, CTA 0
 // finds the k-th key by an exact radix select on the remaining 20 bits
 // instead and sorts the k keys. k is at most 16,384.
+// A request served by one CTA (at most 8,192 doc tokens) takes a shorter
+// path first: its keys stay in registers, one histogram gives the k-th key's
+// bucket and where each bucket starts in descending order, and when at most
+// 1,024 keys lie in that bucket or above and ordering them by counting
+// inside their buckets takes at most 131,072 comparisons (the sum of the
+// squared bucket lengths), the keys are staged bucket by bucket and each
+// finds its place by counting the keys of its own bucket before it;
+// otherwise it continues on the path above.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
@@ -35,6 +43,10 @@ static_assert(kTopkMaxK <= kTopkSortMax, "the k selected keys must fit the stagi
 constexpr int kTopkMaxCluster = 8;
 constexpr int kTopkSlice = 8192;     // doc tokens per CTA before the cluster grows
 constexpr int kRankMax = 256;        // longest bucket ordered by counting ranks (longer: sorted)
+constexpr int kLeanKeys = kTopkSlice / kTopkThreads;   // keys per thread on the one-CTA path
+constexpr int kLeanRank = 1024;      // most keys the one-CTA path orders by counting
+constexpr uint32_t kLeanWork = 131072;   // most comparisons (sum of squared bucket lengths) it makes
+static_assert(kLeanKeys * kTopkThreads == kTopkSlice, "one-CTA path: whole keys per thread");
 
 struct TopkSmem {
   uint64_t staged[kTopkSortMax];     // composite keys of the buckets this CTA orders, at their final bucket ranges
@@ -215,6 +227,49 @@ __device__ __forceinline__ void cleaners_in_warp(uint64_t (&r)[E], int st, int l
   }
 }
 
+// Place of each of a[0, m): the keys are grouped by 12-bit bucket in
+// descending bucket order, bucket d ending at end[d] and holding len[d]
+// keys; a key's place is its bucket's start plus the keys of its bucket
+// that sort before it, counted by P threads per key. Keys placed below k are
+// written out.
+__device__ __forceinline__ void rank_in_buckets(const uint64_t* a, int m, const uint32_t* end,
+                                                const uint32_t* len, int k, int32_t* out_idx, float* out_val) {
+  const int tid = threadIdx.x;
+  int P = 32;
+  while (P > 1 && m * P > kTopkThreads) P >>= 1;
+  const int per_pass = kTopkThreads / P;
+  const int p_lane = tid & (P - 1);
+  for (int f0 = 0; f0 < m; f0 += per_pass) {
+    const int f = f0 + tid / P;
+    uint64_t me = 0ull;
+    int first = 0, n_b = 0;
+    if (f < m) {
+      me = a[f];
+      const uint32_t d = (~uint32_t(me >> 32)) >> 20;
+      n_b = int(len[d]);
+      first = int(end[d]) - n_b;
+    }
+    const uint64_t* run = a + first;
+    int c[4] = {0, 0, 0, 0};
+    int j = p_lane;
+    for (; j + 3 * P < n_b; j += 4 * P) {   // four independent loads in flight per step
+      uint64_t v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = run[j + u * P];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) c[u] += v[u] < me ? 1 : 0;
+    }
+    for (; j < n_b; j += P) c[0] += run[j] < me ? 1 : 0;
+    int cnt = (c[0] + c[1]) + (c[2] + c[3]);
+    for (int o = 1; o < P; o <<= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    const int place = first + cnt;
+    if (f < m && p_lane == 0 && place < k) {
+      out_idx[place] = int32_t(me & 0xffffffffu);
+      if (out_val) out_val[place] = __uint_as_float(~uint32_t(me >> 32));
+    }
+  }
+}
+
 // The whole CTA sorts a[0, len), len <= 1024 * E; steps whose partners are
 // in another warp go through shared memory between block barriers.
 template <int E>
@@ -327,6 +382,51 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     }
   }
   if (k == 0) return;   // the whole cluster leaves together
+
+  if (csize == 1) {
+    // One CTA: the request's keys (at most 8,192) in registers, one histogram
+    // of the 12-bit buckets, the k-th key's bucket d1; the keys of d1 and of
+    // the buckets above it, when there are at most 1,024, are ordered by
+    // counting. Otherwise the general path below runs.
+    uint32_t u[kLeanKeys];
+#pragma unroll
+    for (int j = 0; j < kLeanKeys; ++j) {
+      const int i = j * kTopkThreads + tid;
+      u[j] = i < n ? impact_key(__ldg(keys + i)) : 0u;
+    }
+    for (int i = tid; i < kTopkBins; i += kTopkThreads) S.hist[i] = 0;
+    if (tid == 0) S.cnt[0] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kLeanKeys; ++j)
+      if (j * kTopkThreads + tid < n) atomicAdd(&S.hist[u[j] >> 20], 1u);
+    __syncthreads();
+    // S.cursor[d]: keys in the buckets above d (where bucket d starts)
+    select_digit(S.hist, kTopkBins, uint32_t(k), S.sel, S.warp_sums, S.cursor);
+    const uint32_t d1 = S.sel[0];
+    const int m = k - int(S.sel[1]) + int(S.hist[d1]);   // keys in d1 and above
+    if (m <= kLeanRank) {
+      // comparisons of the counting: the squared lengths of the buckets from d1 up
+      uint32_t work = 0;
+      for (int d = tid; d < kTopkBins; d += kTopkThreads)
+        if (d >= int(d1)) work += S.hist[d] * S.hist[d];
+      for (int o = 16; o > 0; o >>= 1) work += __shfl_xor_sync(0xffffffffu, work, o);
+      if ((tid & 31) == 0 && work > 0) atomicAdd(&S.cnt[0], work);
+    }
+    __syncthreads();
+    if (m <= kLeanRank && S.cnt[0] <= kLeanWork) {
+      // stage bucket by bucket; afterwards S.cursor[d] is where bucket d ends
+#pragma unroll
+      for (int j = 0; j < kLeanKeys; ++j) {
+        const int i = j * kTopkThreads + tid;
+        if (i < n && (u[j] >> 20) >= d1) S.staged[atomicAdd(&S.cursor[u[j] >> 20], 1u)] = composite(u[j], i);
+      }
+      __syncthreads();
+      rank_in_buckets(S.staged, m, S.cursor, S.hist, k, out_idx, out_val);
+      return;
+    }
+    __syncthreads();   // every thread has read S.hist and S.sel before the general path rewrites them
+  }
 
 
   // Pass 1: histogram of the 12-bit buckets (sign, exponent, 3 mantissa bits)

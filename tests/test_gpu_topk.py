@@ -126,3 +126,31 @@ def test_whole_sort_boundary():
     # 4,096 doc tokens are sorted whole by one CTA; 4,097 take the bucket path
     rng = np.random.default_rng(12)
     check([rng.random(4096), rng.lognormal(-4, 1.0, 4097), rng.integers(0, 3, 4096).astype(np.float64)], 0.15)
+
+
+def test_one_cta_counting_limits():
+    # A request of at most 8,192 doc tokens is ordered by counting inside its
+    # 12-bit buckets when at most 1,024 keys lie in the k-th key's bucket or
+    # above and their squared bucket lengths add up to at most 131,072;
+    # otherwise it takes the general path. The top keys are drawn inside
+    # chosen buckets (fp32 bit patterns with fixed top 12 bits, from 2.0 up),
+    # the rest below 0.5; k takes all top keys but one.
+    rng = np.random.default_rng(13)
+    low = 0.5 * rng.random(3000)
+
+    def buckets(sizes):
+        parts = [((np.uint32(1024 + j) << np.uint32(20)) | rng.integers(0, 1 << 20, c).astype(np.uint32))
+                 for j, c in enumerate(sizes)]
+        return np.concatenate(parts).view(np.float32).astype(np.float64)
+
+    for sizes in ([256, 147, 147, 149],        # 131,019 comparisons: counting
+                  [256, 147, 147, 150],        # 131,254: general path
+                  [64] * 16,                   # 1,024 keys: counting
+                  [64] * 15 + [65],            # 1,025 keys (65,665 comparisons): general path
+                  [362], [363],                # one bucket: 131,044 counting, 131,769 general
+                  [40, 3, 100, 0, 77]):        # short buckets
+        top = buckets(sizes)
+        seg = np.concatenate([low[:1500], top, low[1500:]])
+        check([seg], (len(top) - 0.5) / len(seg))
+    tied = np.concatenate([low, np.full(200, 1.0), low[:100]])
+    check([tied, rng.random(7000)], 0.05)           # 200 equal keys above the rest; uniform keys
