@@ -102,7 +102,7 @@ def _code_only(text: str) -> str:
 
 # the source file of each timed kernel kind; its digest also covers the
 # device-side headers every kernel includes
-KERNEL_SOURCE = {"attn": "attn_fwd.cu", "combine": "attn_fwd.cu", "impact": "impact.cu", "topk": "topk.cu",
+KERNEL_SOURCE = {"attn": "attn_fwd.cu", "combine": "attn_combine.cu", "impact": "impact.cu", "topk": "topk.cu",
                  "rc_gemm": "recompute.cu", "rc_copy": "recompute.cu", "rc_plan": "recompute.cu",
                  "kv_decode": "kv_decode.cu", "simt_attn": "simt_f32.cu", "simt_impact": "simt_f32.cu"}
 
