@@ -230,7 +230,7 @@ static Plan plan_split_uncached(const rag_batch& b, int num_kv_heads, int group,
   // attention unit of one Q tile (at most 128 rows: decode steps, one query
   // head per KV head) runs its tiles faster (two S buffers, one softmax
   // warpgroup), so its fixed cost is more tiles' worth: 4 beats 2 by 15 % on
-  // the 16-request decode step.
+  // the 16-request decode step, and 3 (7 % slower) and 8 (30 % slower) there.
   const bool one_q_tile = what == PlanFor::kAttention && avg_q * group <= kBM;
   const double kItemOverheadTiles = one_q_tile ? 4.0 : 2.0;
   const double total_tiles = units * tiles_avg;
