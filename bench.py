@@ -102,7 +102,7 @@ def _code_only(text: str) -> str:
 
 # the source file of each timed kernel kind; its digest also covers the
 # device-side headers every kernel includes
-KERNEL_SOURCE = {"attn": "attn_fwd.cu", "combine": "attn_combine.cu", "impact": "impact.cu", "topk": "topk.cu",
+KERNEL_SOURCE = {"attn": "attn_fwd.cu", "attn_dec": "decode_fwd.cu", "combine": "attn_combine.cu", "impact": "impact.cu", "topk": "topk.cu",
                  "rc_gemm": "recompute.cu", "rc_copy": "recompute.cu", "rc_plan": "recompute.cu",
                  "kv_decode": "kv_decode.cu", "simt_attn": "simt_f32.cu", "simt_impact": "simt_f32.cu"}
 
@@ -328,6 +328,7 @@ def run_gpu(args, w, rank, world, device):
     avg_s = dom_ms / dom_n / 1e3
     per_launch = {
         "attn": (work["attn_flops_per_launch"], work["attn_bytes_per_launch"]),
+        "attn_dec": (work["attn_flops_per_launch"], work["attn_bytes_per_launch"]),
         "combine": (0, 0),
         "impact": (work["impact_flops_per_launch"], work["impact_bytes_per_launch"]),
         "topk": (0, (lay.total_doc + lay.total_q) * 4),

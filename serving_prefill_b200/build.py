@@ -19,7 +19,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librag.so")
-SOURCES = ["rag_api.cu", "attn_fwd.cu", "attn_combine.cu", "impact.cu", "topk.cu", "simt_f32.cu", "pool_write.cu", "rag_static.cu", "selftest.cu", "recompute.cu", "kv_decode.cu"]
+SOURCES = ["rag_api.cu", "attn_fwd.cu", "attn_combine.cu", "decode_fwd.cu", "impact.cu", "topk.cu", "simt_f32.cu", "pool_write.cu", "rag_static.cu", "selftest.cu", "recompute.cu", "kv_decode.cu"]
 HEADERS = ["ptx.cuh", "common.cuh", "params.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

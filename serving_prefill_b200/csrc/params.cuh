@@ -246,6 +246,10 @@ cudaError_t launch_attn_fwd(const CUtensorMap&, const CUtensorMap&, const CUtens
 cudaError_t launch_attn_combine(const CombineParams&, int max_rb, int max_block_rows, int num_requests,
                                 cudaStream_t);
 cudaError_t launch_rope_table(const BatchDev&, double base, float2* table, cudaStream_t);
+// attention for query blocks of at most 16 rows (tq: a Q map whose box is those 16 rows)
+cudaError_t launch_decode_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const CUtensorMap& tkq, const CUtensorMap& tvq, const FwdParams& p, int grid,
+                               cudaStream_t stream);
 cudaError_t launch_impact(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const ImpactParams&, int,
                           cudaStream_t);
 cudaError_t launch_topk(const TopkParams&, int, int, cudaStream_t);

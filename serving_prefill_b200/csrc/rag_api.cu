@@ -25,7 +25,7 @@ constexpr int kRcMinDModel = 64;
 // ------------------------------------------------------------ profiling
 
 enum Kind { kKindPoolWrite = 0, kKindAttn, kKindCombine, kKindImpact, kKindTopk, kKindSimtAttn, kKindSimtImpact,
-            kKindRcPlan, kKindRcCopy, kKindRcGemm, kKindRope, kKindKvDecode, kNumKinds };
+            kKindRcPlan, kKindRcCopy, kKindRcGemm, kKindRope, kKindKvDecode, kKindDecAttn, kNumKinds };
 
 struct ProfRecord {
   int kind;
@@ -469,7 +469,10 @@ static rag_status fused_prefill(const rag_kv_pool* pool, int32_t layer, const ra
   const int H_kv = pool->num_kv_heads;
   const uint64_t pool_rows = uint64_t(pool->num_layers) * pool->num_pages * H_kv * kPage;
 
-  CUtensorMap tm_q, tm_k, tm_v, tm_kq, tm_vq;
+  // query blocks of at most 16 rows (decode steps) take the transposed kernel
+  // of decode_fwd.cu: a key per thread instead of a row per thread
+  const bool use_dec = rope_base <= 0.0 && int64_t(b.max_q) * G <= 16 && 16 % G == 0;
+  CUtensorMap tm_q, tm_qd, tm_k, tm_v, tm_kq, tm_vq;
   {
     const uint64_t dq[3] = {uint64_t(kHeadDim), uint64_t(num_q_heads), uint64_t(b.total_q)};
     const uint64_t sq[2] = {uint64_t(kHeadDim) * 2, uint64_t(num_q_heads) * kHeadDim * 2};
@@ -484,6 +487,9 @@ static rag_status fused_prefill(const rag_kv_pool* pool, int32_t layer, const ra
         !make_map(&tm_v, pool->v, 2, dp, sp, bp) || !make_map(&tm_kq, kq, 3, dk, sk, bk) ||
         !make_map(&tm_vq, vq, 3, dk, sk, bk))
       return RAG_ERR_CUDA;
+    // the decode kernel's Q box is its 16 rows: G query heads of 16 / G tokens
+    const uint32_t bqd[3] = {64u, uint32_t(G), uint32_t(use_dec ? 16 / G : 1)};
+    if (use_dec && !make_map(&tm_qd, q, 3, dq, sq, bqd)) return RAG_ERR_CUDA;
   }
   float* row_m2 = reinterpret_cast<float*>(ws + wl.off_m2);
   float* row_il = reinterpret_cast<float*>(ws + wl.off_il);
@@ -521,8 +527,9 @@ static rag_status fused_prefill(const rag_kv_pool* pool, int32_t layer, const ra
   fp.max_items = pf.max_items;
   fp.rope = rope;
   {
-    LaunchScope ls(kKindAttn, s);
-    cudaError_t e = launch_attn_fwd(tm_q, tm_k, tm_v, tm_kq, tm_vq, fp, pf.grid, s);
+    LaunchScope ls(use_dec ? kKindDecAttn : kKindAttn, s);
+    cudaError_t e = use_dec ? launch_decode_attn(tm_qd, tm_k, tm_v, tm_kq, tm_vq, fp, pf.grid, s)
+                            : launch_attn_fwd(tm_q, tm_k, tm_v, tm_kq, tm_vq, fp, pf.grid, s);
     ls.done(e);
     if (e != cudaSuccess) return RAG_ERR_CUDA;
   }

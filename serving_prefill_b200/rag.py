@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librag.so")
 RAG_BF16, RAG_F32 = 0, 1
 PAGE_SIZE = 16
 KERNEL_KINDS = ("pool_write", "attn", "combine", "impact", "topk", "simt_attn", "simt_impact", "rc_plan", "rc_copy",
-                "rc_gemm", "rope_table", "kv_decode")
+                "rc_gemm", "rope_table", "kv_decode", "attn_dec")
 
 STATUS = {
     0: "ok", 1: "invalid argument", 2: "inconsistent shape", 3: "page id outside the pool",
