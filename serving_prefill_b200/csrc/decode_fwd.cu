@@ -9,8 +9,9 @@
 // so that a thread owns a key instead of a row:
 //   S^T = K Q^T   (tcgen05, A = K tile [128 keys x 128 d], B = Q [16 rows])
 //   per row: max over the 128 keys by warp shuffles and a shared exchange
-//   between the four key warps, 16 exponentials per thread,
-//   P^T (fp16, [16 rows x 128 keys]) written to shared memory,
+//   between the four key warps, one exponential per row and thread, the rows
+//   padded to R = 4, 8 or 16 (compiled for each; a decode step with G = 4
+//   has 4), P^T (fp16, [16 rows x 128 keys]) written to shared memory,
 //   O^T += V^T P^T (A = the V tile read as [d x keys], B = P^T)
 // O^T sits in TMEM with d on the lanes; the epilogue writes the same partial
 // rows (O/l in fp16, m, l) or output rows as the prefill kernel, so the split
