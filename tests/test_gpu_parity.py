@@ -44,8 +44,14 @@ def small_cases():
         "one_query_token": scaled(l2, num_q_heads=8, num_kv_heads=8, chunk_lens=(1, 15, 16, 17, 129), q_len=1),
         "query_longer_than_tile": scaled(l3, num_layers=1, num_q_heads=4, num_kv_heads=2, chunk_lens=(60,),
                                          q_len=300),
-        # over 117 requests: the attention kernel's V tiles are double- rather
-        # than triple-buffered (the request table takes the shared memory)
+        # query blocks of at most 16 rows take the decode kernel: 16 rows of
+        # 4 causal query tokens, 10 rows of 5 tokens (padded to 16), and a
+        # batch whose items pad to 4, 8 or 16 rows
+        "short_query_g4": scaled(l3, num_layers=1, num_q_heads=8, num_kv_heads=2, chunk_lens=(300, 77, 1), q_len=4),
+        "short_query_g2": scaled(l3, num_layers=1, num_q_heads=4, num_kv_heads=2, chunk_lens=(129, 16, 200), q_len=5),
+        "short_queries_batched": scaled(b16, num_q_heads=8, num_kv_heads=2, n_requests=5, n_pool_chunks=6,
+                                        chunk_len_range=(1, 300), chunks_per_req=(1, 3), q_range=(1, 4)),
+        # many requests: one prefix entry per request in the kernels' shared memory
         "many_requests": scaled(b16, num_q_heads=8, num_kv_heads=2, n_requests=130, n_pool_chunks=40,
                                 chunk_len_range=(1, 300), chunks_per_req=(1, 3), q_range=(1, 40)),
     }
