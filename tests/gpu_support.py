@@ -22,7 +22,9 @@ TIE_RTOL = 1e-4
 class DeviceCase:
     """A workload's pool (the given layers), batch and engine on the GPU."""
 
-    def __init__(self, w, lay=None, layers=None, device="cuda", spare_pages=0):
+    def __init__(self, w, lay=None, layers=None, device="cuda", spare_pages=0, transform=None):
+        """transform(inputs): optional in-place change of each layer's seeded
+        inputs before they are written; the oracle sees the same inputs."""
         self.w = w
         self.lay = make_layout(w) if lay is None else lay
         self.layers = list(range(w.num_layers)) if layers is None else list(layers)
@@ -37,6 +39,8 @@ class DeviceCase:
         pages = [p.to(torch.int32).to(device) for p in self.lay.chunk_pages]
         for layer in self.layers:
             inp = make_layer_inputs(w, self.lay, layer)
+            if transform is not None:
+                transform(inp)
             self.inputs[layer] = inp
             write_chunks(self.pool, layer, pages, [k.to(device) for k in inp.chunk_k],
                          [v.to(device) for v in inp.chunk_v], device_err=self.err)

@@ -69,6 +69,27 @@ def test_parity_small(name):
         check_layer(case, layer, with_impact=(layer == w.impact_layer_index))
 
 
+def _keys_growing_by_chunk(inp):
+    # chunk c's keys times 4^c (exact in bf16): along a request's keys the row
+    # maxima jump by many 2^8 steps, so O is rescaled in the middle of rows
+    for c, k in enumerate(inp.chunk_k):
+        k.mul_(float(4 ** (c % 4)))
+
+
+@pytest.mark.parametrize("name", ["decode_kernel", "prefill_kernel"])
+def test_rescale_when_row_maxima_grow(name):
+    w = {
+        # 4 rows per unit: the decode kernel
+        "decode_kernel": scaled(get_workload("decode16"), num_q_heads=8, num_kv_heads=2, n_requests=3, n_pool_chunks=4,
+                                chunk_len_range=(150, 400), chunks_per_req=(3, 4), context_range=(1, 40)),
+        # 80 rows per unit: the prefill kernel
+        "prefill_kernel": scaled(get_workload("llama3_8b_l32"), num_layers=1, num_q_heads=8, num_kv_heads=2,
+                                 chunk_lens=(200, 256, 300, 180), q_len=20),
+    }[name]
+    case = DeviceCase(w, layers=[0], transform=_keys_growing_by_chunk)
+    check_layer(case, 0, with_impact=(w.impact_layer_index == 0))
+
+
 @pytest.mark.parametrize("name", ["tiny", "pooled", "gqa4_rows3"])
 def test_pool_write_bit_exact(name):
     w = CASES[name]
