@@ -27,9 +27,15 @@ pytestmark = pytest.mark.gpu
 RAG_ERR_PAGE_OOB, RAG_ERR_TIMEOUT, RAG_ERR_GEOMETRY, RAG_ERR_RANGE = 3, 6, 8, 9
 
 
-def pooled():
+def pooled(path="prefill"):
+    """Four requests over a shared chunk pool; path "decode" gives them 1-4
+    query tokens (at most 16 rows per unit), so the decode kernel runs."""
+    q_range = (1, 4) if path == "decode" else (5, 60)
     return scaled(get_workload("batched16"), num_q_heads=8, num_kv_heads=2, n_requests=4, n_pool_chunks=8,
-                  chunk_len_range=(20, 300), chunks_per_req=(2, 3), q_range=(5, 60))
+                  chunk_len_range=(20, 300), chunks_per_req=(2, 3), q_range=q_range)
+
+
+PATHS = ["prefill", "decode"]
 
 
 def host_arrays(lay):
@@ -66,8 +72,9 @@ def check_other_requests(case, out, ref, skip):
         at += nd + ql
 
 
-def test_page_outside_the_pool_is_skipped_and_reported():
-    w = pooled()
+@pytest.mark.parametrize("path", PATHS)
+def test_page_outside_the_pool_is_skipped_and_reported(path):
+    w = pooled(path)
     case = DeviceCase(w, layers=[0])
     ref = case.oracle(0, True)
     arrays = host_arrays(case.lay)
@@ -82,8 +89,9 @@ def test_page_outside_the_pool_is_skipped_and_reported():
     assert len(set(out["topk_idx"][0][:k0].tolist())) == k0
 
 
-def test_chunk_with_one_page_too_many_is_reported_and_exact():
-    w = pooled()
+@pytest.mark.parametrize("path", PATHS)
+def test_chunk_with_one_page_too_many_is_reported_and_exact(path):
+    w = pooled(path)
     case = DeviceCase(w, layers=[0])
     ref = case.oracle(0, True)
     rc, cd, cp, pid, qo = host_arrays(case.lay)
@@ -98,8 +106,9 @@ def test_chunk_with_one_page_too_many_is_reported_and_exact():
     check_other_requests(case, out, ref, skip=-1)    # every request, the altered one included
 
 
-def test_chunk_with_one_page_too_few_is_reported():
-    w = pooled()
+@pytest.mark.parametrize("path", PATHS)
+def test_chunk_with_one_page_too_few_is_reported(path):
+    w = pooled(path)
     case = DeviceCase(w, layers=[0])
     ref = case.oracle(0, True)
     rc, cd, cp, pid, qo = host_arrays(case.lay)
@@ -137,14 +146,17 @@ def test_v_beyond_the_fp16_range_is_reported_by_the_pool_write(value, flagged):
     check_layer(case, 0, with_impact=True)
 
 
-def test_v_q_beyond_the_fp16_range_is_reported_by_the_attention():
+@pytest.mark.parametrize("path", PATHS)
+def test_v_q_beyond_the_fp16_range_is_reported_by_the_attention(path):
     """The query block's own V_q enters the product as fp16 too: a value of
     70,000 is saturated and the call reports RAG_ERR_RANGE; the rest of the
-    output keeps parity with the oracle, which saturates it the same way."""
-    w = scaled(get_workload("llama2_7b_l1"), num_q_heads=4, num_kv_heads=4, chunk_lens=(200, 77), q_len=20)
+    output keeps parity with the oracle, which saturates it the same way
+    (a 4-token query block takes the decode kernel)."""
+    q_len = 4 if path == "decode" else 20
+    w = scaled(get_workload("llama2_7b_l1"), num_q_heads=4, num_kv_heads=4, chunk_lens=(200, 77), q_len=q_len)
     case = DeviceCase(w, layers=[0])
     inp = case.inputs[0]
-    inp.vq[7, 2, 100] = 70000.0
+    inp.vq[min(7, q_len - 1), 2, 100] = 70000.0
     case.dev_inputs[0] = (inp.q.cuda(), inp.kq.cuda(), inp.vq.cuda())
     out = case.run_layer(0, with_impact=True)
     ref = case.oracle(0, True)
