@@ -32,10 +32,13 @@ def _cases():
                          chunk_len_range=(1, 400), chunks_per_req=(1, 4), q_range=(1, 90)),
         # long key range: split-KV partials in the scratch array, then the combine
         "split": scaled(l70, num_q_heads=16, num_kv_heads=2, chunk_lens=(2048,) * 6, q_len=150),
+        # decode step (one token, 4 rows per unit): the decode kernel
+        "decode": scaled(get_workload("decode16"), num_q_heads=8, num_kv_heads=2, n_requests=6, n_pool_chunks=10,
+                         chunk_len_range=(100, 900), chunks_per_req=(2, 4), context_range=(1, 200)),
     }
 
 
-@pytest.mark.parametrize("name", ["pooled", "split"])
+@pytest.mark.parametrize("name", ["pooled", "split", "decode"])
 def test_static_scratch_matches_workspace_entry(name):
     w = _cases()[name]
     case = DeviceCase(w, layers=[0])
