@@ -391,7 +391,8 @@ RAG_API int64_t rag_launch_count(void);
  * milliseconds and launch counts per kernel kind (0 pool write, 1 attention,
  * 2 split combine, 3 impact, 4 top-k, 5 fp32 attention, 6 fp32 impact,
  * 7 recompute plan, 8 recompute page copy, 9 recompute projection,
- * 10 RoPE table, 11 KV decode) into
+ * 10 RoPE table, 11 KV decode, 12 attention of query blocks of at most 16
+ * rows, e.g. decode steps) into
  * the first n_kinds entries of ms and launches (either may be NULL), and
  * resets the record. */
 RAG_API void rag_profile_enable(int32_t on);
